@@ -1,0 +1,80 @@
+"""Planted mistakes in the oracle must be caught by its pins (CPU only).
+
+Each case swaps one oracle function for a plausible wrong variant (a dropped
+term, a wrong index, a transposed operand, a wrong tie-break) on the CPU and
+checks that at least one pin in test_oracle_pins.py then fails.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import attention as oatt
+from oracle import blocksel as obi
+from oracle import decode as odec
+from oracle import vslash as ovs
+import tests.test_oracle_pins as pins
+
+
+def _sum_pool(x, block=64):
+    n, d = x.shape[-2], x.shape[-1]
+    return np.asarray(x, dtype=np.float64).reshape(x.shape[:-2] + (n // block, block, d)).sum(axis=-2)
+
+
+def _transposed_scores(qbar, kbar):
+    return kbar @ qbar.T
+
+
+def _no_causal_rows(q_rows, row_ids, k, v, blocks, cols, scale):
+    keys = oatt._key_set(blocks, cols)
+    Z = (q_rows @ k[keys].T) * scale
+    m = Z.max(axis=1, keepdims=True)
+    P = np.exp(Z - m)
+    l = P.sum(axis=1, keepdims=True)
+    return (P @ v[keys]) / l, (m + np.log(l))[:, 0]
+
+
+def _unscaled_rows(q_rows, row_ids, k, v, blocks, cols, scale):
+    return oatt.__dict__["_orig_rows"](q_rows, row_ids, k, v, blocks, cols, 1.0)
+
+
+def _high_tie_select(scores, cand, e):
+    if e <= 0 or cand.size == 0:
+        return np.zeros(0, dtype=np.int64)
+    order = np.lexsort((-cand, -scores))
+    return np.sort(cand[order[:e]])
+
+
+def _slash_plus(q, k, last_q, scale, heads=None):
+    vert, slash = ovs.__dict__["_orig_vs"](q, k, last_q, scale, heads)
+    return vert, {h: np.roll(s, 1) for h, s in slash.items()}
+
+
+@pytest.mark.parametrize("case", ["sum_pool", "transposed", "no_causal", "unscaled", "high_tie", "slash_shift"])
+def test_planted_mistake_is_caught(case, monkeypatch):
+    if case == "sum_pool":
+        monkeypatch.setattr(oracle, "pool_blocks", _sum_pool)
+        monkeypatch.setattr(obi, "pool_blocks", _sum_pool)
+        checks = [pins.test_pooled_score_commutes_with_matmul]
+    elif case == "transposed":
+        monkeypatch.setattr(oracle, "block_scores", _transposed_scores)
+        monkeypatch.setattr(obi, "block_scores", _transposed_scores)
+        checks = [pins.test_pooled_score_commutes_with_matmul]
+    elif case == "no_causal":
+        monkeypatch.setattr(oatt, "sparse_attention_rows", _no_causal_rows)
+        checks = [pins.test_all_blocks_equals_dense_causal_sdpa]
+    elif case == "unscaled":
+        monkeypatch.setitem(oatt.__dict__, "_orig_rows", oatt.sparse_attention_rows)
+        monkeypatch.setattr(oatt, "sparse_attention_rows", _unscaled_rows)
+        checks = [pins.test_all_blocks_equals_dense_causal_sdpa]
+    elif case == "high_tie":
+        monkeypatch.setattr(oracle, "select_top", _high_tie_select)
+        monkeypatch.setattr(odec, "select_top", _high_tie_select)
+        checks = [pins.test_select_top_matches_python_sort, pins.test_decode_zero_query_keeps_lowest_blocks]
+    else:
+        monkeypatch.setitem(ovs.__dict__, "_orig_vs", ovs.vs_scores)
+        monkeypatch.setattr(oracle, "vs_scores", _slash_plus)
+        checks = [pins.test_vs_scores_closed_form_uniform]
+    for chk in checks:
+        with pytest.raises(AssertionError):
+            chk()
