@@ -1,0 +1,436 @@
+"""Benchmark of the dynamic-sparse-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-decode] [--no-e2e] [--no-cpu-baseline]
+
+A step is one prefill layer of the block-sparse path on the named workload
+(default: the LLaMA-3-8B-shaped layer at 128K tokens, 32 q-heads / 8 KV
+heads, d=128, keep 10% of causal blocks plus sink and diagonal): the block
+index (sparse_index_estimate) followed by causal block-sparse attention
+(block_sparse_attn_fwd), with inputs resident in HBM.  The metric is the
+effective TFLOP/s counting only the FLOPs of the selected blocks (diagonal
+blocks at their causal 2080 of 4096 elements); ms_per_step is ms per layer.
+The sparse decode GB/s (batch 16, 128K cache, keep 512 + the last block) is
+reported beside it under "decode".
+
+One JSON line is printed by rank 0.  Multi-GPU (torchrun): every rank runs its
+own independent layer (weak scaling, no data-path collective); timing is the
+max over ranks of the device time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "block-sparse prefill effective TFLOP/s at 128K (selected-block FLOPs)"
+UNIT = "TFLOP/s"
+DIAG_ELEMS = 64 * 65 // 2
+
+
+def prefill_flops(block_cnt: torch.Tensor, d: int) -> float:
+    """Selected-block FLOPs: 4*64*64*d per off-diagonal block (QK^T and PV), the
+    diagonal block at its 2080 causal elements.  Every block-sparse row holds its
+    diagonal block."""
+    cnt = block_cnt.to(torch.float64)
+    return float(((cnt - 1).clamp(min=0) * 4 * 64 * 64 * d + 4 * DIAG_ELEMS * d).sum().item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, maxmhz, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                maxmhz = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": maxmhz, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": maxmhz, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def dist_setup(ngpus: int):
+    if ngpus <= 1 and "RANK" not in os.environ:
+        return 0, 1, 0
+    import datetime
+
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local):
+    import dynamic_sparse_attention_03_b200 as dsa
+
+    dsa.load_library()
+    dev = torch.device("cuda", local)
+    p = synth.CONFIGS[args.workload]
+    w = synth.make_prefill(args.workload, device=dev, seed=p["seed"] + 1000 * rank)
+    Hq, n, d = w.q.shape
+    kf, rho = p.get("k_fixed", 0), p.get("keep_ratio", 0.0)
+    kcap = dsa.block_index_capacity(n, kf, rho)
+    bi = torch.empty((Hq, n // 64, kcap), dtype=torch.int32, device=dev)
+    bc = torch.empty((Hq, n // 64), dtype=torch.int32, device=dev)
+    o = torch.empty_like(w.q)
+    ws = dsa.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        dsa.sparse_index_estimate(w.q, w.k, k_fixed=kf, keep_ratio=rho, kcap=kcap, block_idx=bi, block_cnt=bc, ws=ws)
+        dsa.block_sparse_attn_fwd(w.q, w.k, w.v, bi, bc, out=o, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flops = prefill_flops(bc, d)
+    launches_per_step = 5 if Hq * (n // 64) ** 2 * 4 <= (1 << 30) else None
+    # timed region
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        # the attention kernel alone, same stream, for the roofline
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        i0, i1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(2, min(args.steps, 5))
+        i0.record(stream)
+        for _ in range(reps):
+            dsa.sparse_index_estimate(w.q, w.k, k_fixed=kf, keep_ratio=rho, kcap=kcap, block_idx=bi, block_cnt=bc,
+                                      ws=ws)
+        i1.record(stream)
+        a0.record(stream)
+        for _ in range(reps):
+            dsa.block_sparse_attn_fwd(w.q, w.k, w.v, bi, bc, out=o, ws=ws)
+        a1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms, world)
+    attn_ms = a0.elapsed_time(a1) / reps
+    index_ms = i0.elapsed_time(i1) / reps
+    status = dsa.get_status(ws)
+    value = flops * world / (ms * 1e-3) / 1e12
+    peaks, src = load_peaks()
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    density = float(bc.to(torch.float64).sum().item()) / (Hq * (n // 64) * (n // 64 + 1) / 2)
+    res = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "Hq": Hq, "Hkv": w.k.shape[0], "seq_len": n, "head_dim": d,
+                   "keep": f"k_fixed={kf}" if kf else f"ratio={rho}+sink+diag", "block": 64,
+                   "selected_block_density": round(density, 5),
+                   "l2": "inputs larger than L2 (Q 1.07 GB, K/V 268 MB each at 128K), no flush",
+                   "parallelism": f"independent layer per GPU x{world}"},
+        "breakdown_ms": {"index": round(index_ms, 4), "attention": round(attn_ms, 4)},
+        "effective_flops_per_step": flops,
+        "roofline": {"bound": "tensor", "kernel": "bsa_fwd_kernel<128>", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{src} bf16_tflops_sustained"},
+        "clocks": clk.summary(),
+        "gpu_launches": (launches_per_step * args.steps) if launches_per_step else None,
+        "device_status": status,
+    }
+    return res, (w, bi, bc, kf, rho, kcap, flops, ws)
+
+
+def run_decode(args, local):
+    import dynamic_sparse_attention_03_b200 as dsa
+
+    dev = torch.device("cuda", local)
+    dw = synth.make_decode("decode-b16-128k", device=dev)
+    p = dw.params
+    cent = dsa.pool_keys(dw.k_cache)
+    ws = dsa.Workspace(dev)
+    o, si, sc = dsa.sparse_decode_attn(dw.q, dw.k_cache, dw.v_cache, cent, keep=p["keep"], return_sel=True, ws=ws)
+    torch.cuda.synchronize()
+    # union of the GQA group's kept blocks: each K/V block read once per (b, KV head)
+    B, Hq, dd = dw.q.shape
+    Hkv, S = dw.k_cache.shape[1], dw.k_cache.shape[2]
+    nb = S // 64
+    grp = Hq // Hkv
+    mask = torch.zeros((B, Hkv, nb), dtype=torch.bool, device=dev)
+    for h in range(Hq):
+        idx = si[:, h].long().clamp(min=0)
+        valid = torch.arange(si.shape[-1], device=dev)[None, :] < sc[:, h:h + 1]
+        m2 = torch.zeros((B, nb), dtype=torch.long, device=dev)
+        m2.scatter_add_(1, idx * valid, valid.long())
+        m2 = m2 > 0
+        mask[:, h // grp] |= m2
+    union_blocks = int(mask.sum().item())
+    bytes_kv = union_blocks * 2 * 64 * dd * 2
+    bytes_cent = B * Hkv * nb * dd * 4
+    bytes_io = 2 * B * Hq * dd * 2
+    total = bytes_kv + bytes_cent + bytes_io
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        dsa.sparse_decode_attn(dw.q, dw.k_cache, dw.v_cache, cent, keep=p["keep"], out=o, ws=ws)
+    torch.cuda.synchronize()
+    reps = 20
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        dsa.sparse_decode_attn(dw.q, dw.k_cache, dw.v_cache, cent, keep=p["keep"], out=o, ws=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    dsa.pool_keys(dw.k_cache, out=cent, ws=ws)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    peaks, src = load_peaks()
+    gbs = total / (ms * 1e-3) / 1e9
+    cent_ms = c0.elapsed_time(c1)
+    cent_gbs = (B * Hkv * S * dd * 2 + bytes_cent) / (cent_ms * 1e-3) / 1e9
+    del dw
+    return {"workload": "decode-b16-128k", "ms": round(ms, 4), "GB/s": round(gbs, 1),
+            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": total,
+            "union_kv_blocks": union_blocks, "centroid_build_ms": round(cent_ms, 4),
+            "centroid_build_GB/s": round(cent_gbs, 1), "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": src}
+
+
+def run_e2e(args, ctx, local):
+    """Same metric through the public API with host buffers: pinned host Q/K/V
+    copied in, index + attention, O copied out, every step."""
+    import dynamic_sparse_attention_03_b200 as dsa
+
+    w, bi, bc, kf, rho, kcap, flops, ws = ctx
+    dev = torch.device("cuda", local)
+    hq, hk, hv = (t.to("cpu").pin_memory() for t in (w.q, w.k, w.v))
+    ho = torch.empty_like(hq).pin_memory()
+    dq, dk, dv, do = (torch.empty_like(w.q), torch.empty_like(w.k), torch.empty_like(w.v), torch.empty_like(w.q))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dsa.sparse_index_estimate(dq, dk, k_fixed=kf, keep_ratio=rho, kcap=kcap, block_idx=bi, block_cnt=bc, ws=ws)
+        dsa.block_sparse_attn_fwd(dq, dk, dv, bi, bc, out=do, ws=ws)
+        ho.copy_(do, non_blocking=True)
+
+    steps = max(2, min(args.steps, 5))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size()
+    return {"value": round(flops / (ms * 1e-3) / 1e12, 3), "unit": UNIT, "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+# ------------------------------------------------------------------ CPU oracle (reference arm and cpu_baseline)
+
+def oracle_sample(workload: str, budget_s: float, w=None, seed_rank: int = 0):
+    """Time the fp64 oracle on a bounded sample of the workload: the full block
+    index of one q-head plus the attention of sampled query blocks of that head.
+    Returns (effective TFLOP/s of the sample, description, seconds, cores)."""
+    import oracle
+
+    p = synth.CONFIGS[workload]
+    if w is None:
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        w = synth.make_prefill(workload, device=dev, seed=p["seed"] + 1000 * seed_rank)
+    Hq, n, d = w.q.shape
+    grp = Hq // w.k.shape[0]
+    h = 0
+    q = synth.to_f64(w.q[h:h + 1])
+    k = synth.to_f64(w.k[h // grp:h // grp + 1])
+    v = synth.to_f64(w.v[h // grp:h // grp + 1])
+    kf, rho = p.get("k_fixed", 0), p.get("keep_ratio", 0.0)
+    nqb = n // 64
+    t0 = time.perf_counter()
+    lists, _, _ = oracle.block_index(q, k, k_fixed=kf, keep_ratio=rho)
+    t_index = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    order = [nqb - 1, 0] + rng.permutation(nqb).tolist()
+    flops = 0.0
+    t_att = 0.0
+    items = 0
+    for qb in order:
+        if t_index + t_att > budget_s and items >= 2:
+            break
+        t1 = time.perf_counter()
+        oracle.sparse_attention(q, k, v, lists, None, 1 / math.sqrt(d), items=[(0, qb)])
+        t_att += time.perf_counter() - t1
+        cnt = len(lists[0][qb])
+        flops += (cnt - 1) * 4 * 64 * 64 * d + 4 * DIAG_ELEMS * d
+        items += 1
+    # index cost of one head prorated to the sampled query blocks
+    t_total = t_att + t_index * items / nqb
+    cores = len(os.sched_getaffinity(0))
+    desc = (f"oracle fp64 on host: block index of q-head 0 ({nqb} query blocks, {t_index:.2f}s, prorated) + "
+            f"attention of {items} sampled query blocks of q-head 0")
+    return flops / t_total / 1e12, desc, t_total, cores
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    vals = []
+    desc = ""
+    cores = len(os.sched_getaffinity(0))
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    p = synth.CONFIGS[args.workload]
+    w = synth.make_prefill(args.workload, device=dev, seed=p["seed"])
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup + args.steps):
+        v, desc, secs, cores = oracle_sample(args.workload, budget, w=w)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.mean(vals)
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama3-8b-128k-bs10")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", 0))
+        world = int(os.environ.get("WORLD_SIZE", args.gpus))
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    res, ctx = run_ours(args, rank, world, local)
+    if not args.no_e2e:
+        res["e2e"] = run_e2e(args, ctx, local)
+    if not args.no_decode:
+        res["decode"] = run_decode(args, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, secs, cores = oracle_sample(args.workload, 15.0, w=ctx[0])
+        res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+                               "seconds": round(secs, 2)}
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,449 @@
+// api.cu -- host side of the C ABI declared in include/dsa.h: argument checks,
+// workspace layout, TMA descriptor encoding and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dsa.h"
+#include "attn_fwd.cuh"
+#include "decode.cuh"
+#include "index_kernels.cuh"
+#include "vs_kernels.cuh"
+
+using namespace dsa;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+constexpr size_t kScoreChunkBytes = size_t(1) << 30;   // pooled-score scratch per head chunk
+constexpr int kMaxN = 1 << 21;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct WsCarve {
+  uint8_t* base;
+  size_t off = 0;
+  explicit WsCarve(void* b) : base(static_cast<uint8_t*>(b)) {}
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off = align256(off + bytes);
+    return p;
+  }
+};
+
+int cuda_err(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+int launch_check() { return cuda_err(cudaGetLastError()); }
+
+// Dynamic shared memory above 48 KB needs an opt-in per kernel.
+template <typename K>
+int set_smem(K kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return DSA_OK;
+  return cuda_err(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 2D bf16 view [rows][d] with a 64 x 64 box and 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, int64_t rows, int d) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool validate_env() {
+  const char* v = std::getenv("DSA_VALIDATE");
+  return v && v[0] == '1';
+}
+
+int max_count(int nQB, int k_fixed, int64_t ppm) {
+  int best = 0;
+  for (int i = 0; i < nQB; ++i) {
+    const int c = (i == 0 ? 1 : 2) + extra_budget(i, k_fixed, ppm);
+    best = c > best ? c : best;
+  }
+  return best;
+}
+
+// Device-side list check for block_sparse_attn_fwd in validation mode.
+__global__ void validate_lists_kernel(const int32_t* bidx, const int32_t* bcnt, int kcap, const int32_t* cidx,
+                                      const int32_t* ccnt, int ccap, int nQB, int Hq, uint32_t* status) {
+  const int qb = blockIdx.x, h = blockIdx.y;
+  if (threadIdx.x != 0) return;
+  const size_t row = (size_t)h * nQB + qb;
+  const int nb = bcnt[row];
+  bool bad = nb < 0 || nb > kcap;
+  const int32_t* b = bidx + row * kcap;
+  for (int x = 0; !bad && x < nb; ++x) {
+    if (b[x] < 0 || b[x] > qb) bad = true;
+    if (x > 0 && b[x] <= b[x - 1]) bad = true;
+  }
+  if (!bad && cidx) {
+    const int nc = ccnt[row];
+    if (nc < 0 || nc > ccap) bad = true;
+    const int32_t* c = cidx + row * ccap;
+    int y = 0;
+    for (int x = 0; !bad && x < nc; ++x) {
+      const int j = c[x];
+      if (j < 0 || j >= 64 * qb) bad = true;
+      if (x > 0 && j <= c[x - 1]) bad = true;
+      while (y < nb && b[y] < (j >> 6)) ++y;
+      if (y < nb && b[y] == (j >> 6)) bad = true;
+    }
+  }
+  if (bad) atomicOr(status, kStatusBadList);
+}
+
+template <int D>
+int launch_attn(const void* q, const void* k, const void* v, void* o, int Hq, int Hkv, int n, float scale,
+                const int32_t* bidx, const int32_t* bcnt, int kcap, const int32_t* cidx, const int32_t* ccnt,
+                int ccap, float* lse, uint32_t* status, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, (int64_t)Hq * n, D) || !make_tmap(&tk, k, (int64_t)Hkv * n, D) ||
+      !make_tmap(&tv, v, (int64_t)Hkv * n, D))
+    return DSA_ERR_CUDA;
+  AttnParams p{};
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.block_idx = bidx;
+  p.block_cnt = bcnt;
+  p.col_idx = cidx;
+  p.col_cnt = ccnt;
+  p.status = status;
+  p.kcap = kcap;
+  p.ccap = ccap;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.n = n;
+  p.nQB = n / 64;
+  p.grp = Hq / Hkv;
+  p.npairs = (p.grp + 1) / 2;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const size_t smem = AttnLayout<D>::kSmemAlloc;
+  int rc = set_smem(bsa_fwd_kernel<D>, smem);
+  if (rc) return rc;
+  const int64_t grid = (int64_t)Hkv * p.npairs * p.nQB;
+  bsa_fwd_kernel<D><<<(unsigned)grid, 192, smem, st>>>(tq, tk, tv, p);
+  return launch_check();
+}
+
+template <int D, int G>
+int launch_decode(const DecodeParams& p, int B, int Hkv, int nchmax, size_t sel_smem, cudaStream_t st) {
+  int rc;
+  if ((rc = set_smem(decode_select_kernel<D, G, 256>, sel_smem))) return rc;
+  decode_select_kernel<D, G, 256><<<B * Hkv, 256, sel_smem, st>>>(p);
+  if ((rc = launch_check())) return rc;
+  if ((rc = set_smem(decode_attn_kernel<D, G>, DecLayout<D>::kBytes))) return rc;
+  decode_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 160, DecLayout<D>::kBytes, st>>>(p);
+  return launch_check();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dsa_version(void) { return "dsa 0.1 sm_100a"; }
+
+int dsa_block_index_capacity(int n, int block, int k_fixed, float keep_ratio) {
+  if (n <= 0) return DSA_ERR_INVALID_ARG;
+  if (block != 64 || n % 64 != 0 || n > kMaxN) return DSA_ERR_UNSUPPORTED;
+  const bool fixed = k_fixed > 0, ratio = keep_ratio > 0.f;
+  if (fixed == ratio || !(keep_ratio == keep_ratio) || keep_ratio > 1.0f) return DSA_ERR_INVALID_ARG;
+  const int64_t ppm = ratio ? (int64_t)std::floor((double)keep_ratio * 1e6 + 0.5) : 0;
+  return max_count(n / 64, fixed ? k_fixed : 0, ppm);
+}
+
+int dsa_get_status(const void* ws, dsa_stream_t stream) {
+  if (!ws) return DSA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemsetAsync(const_cast<void*>(ws), 0, sizeof(word), st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (word & kStatusTimeout) return DSA_ERR_TIMEOUT;
+  if (word & kStatusBadList) return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, int d, int block, int k_fixed,
+                          float keep_ratio, int32_t* block_idx, int32_t* block_cnt, int kcap, float* pooled_k,
+                          void* ws, size_t* ws_bytes, dsa_stream_t stream) {
+  if (!k || !ws_bytes || Hkv <= 0 || n <= 0) return DSA_ERR_INVALID_ARG;
+  if (block != 64 || (d != 64 && d != 128) || n % 64 != 0 || n > kMaxN) return DSA_ERR_UNSUPPORTED;
+  if ((int64_t)Hkv * n >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(k) || (q && !aligned16(q))) return DSA_ERR_INVALID_ARG;
+  const int nQB = n / 64;
+  const bool pool_only = (q == nullptr);
+  int64_t ppm = 0;
+  int chunk = 0;
+  if (pool_only) {
+    if (!pooled_k) return DSA_ERR_INVALID_ARG;
+  } else {
+    if (Hq <= 0 || Hq % Hkv != 0 || !block_idx || !block_cnt || kcap <= 0) return DSA_ERR_INVALID_ARG;
+    if ((int64_t)Hq * n >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+    const bool fixed = k_fixed > 0, ratio = keep_ratio > 0.f;
+    if (fixed == ratio || !(keep_ratio == keep_ratio) || keep_ratio > 1.0f) return DSA_ERR_INVALID_ARG;
+    if (ratio) ppm = (int64_t)std::floor((double)keep_ratio * 1e6 + 0.5);
+    if (max_count(nQB, fixed ? k_fixed : 0, ppm) > kcap) return DSA_ERR_CAPACITY;
+    const size_t per_head = (size_t)nQB * nQB * 4;
+    chunk = (int)std::max<size_t>(1, std::min<size_t>((size_t)Hq, kScoreChunkBytes / per_head));
+  }
+  WsCarve c(ws);
+  uint32_t* status = static_cast<uint32_t*>(c.take(kStatusBytes));
+  float* qbar = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hq * nQB * d * 4));
+  float* kbar = pooled_k ? pooled_k : static_cast<float*>(c.take((size_t)Hkv * nQB * d * 4));
+  float* scores = pool_only ? nullptr : static_cast<float*>(c.take((size_t)chunk * nQB * nQB * 4));
+  if (!ws) {
+    *ws_bytes = c.off;
+    return DSA_OK;
+  }
+  if (*ws_bytes < c.off) return DSA_ERR_INVALID_ARG;
+  (void)status;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  if (d == 128) pool_blocks_kernel<128><<<(unsigned)((int64_t)Hkv * nQB), 256, 0, st>>>(kb, kbar, (int64_t)Hkv * nQB);
+  else pool_blocks_kernel<64><<<(unsigned)((int64_t)Hkv * nQB), 256, 0, st>>>(kb, kbar, (int64_t)Hkv * nQB);
+  if (int rc = launch_check()) return rc;
+  if (pool_only) return DSA_OK;
+  const auto* qp = static_cast<const __nv_bfloat16*>(q);
+  if (d == 128) pool_blocks_kernel<128><<<(unsigned)((int64_t)Hq * nQB), 256, 0, st>>>(qp, qbar, (int64_t)Hq * nQB);
+  else pool_blocks_kernel<64><<<(unsigned)((int64_t)Hq * nQB), 256, 0, st>>>(qp, qbar, (int64_t)Hq * nQB);
+  if (int rc = launch_check()) return rc;
+  const int ntr = (nQB + 63) / 64;
+  const unsigned ntiles = (unsigned)(ntr * (ntr + 1) / 2);
+  const size_t sc_smem = 2 * (size_t)d * 64 * 4;
+  const size_t sel_smem = (size_t)nQB * 4;
+  int rc = (d == 128) ? set_smem(block_scores_kernel<128>, sc_smem) : set_smem(block_scores_kernel<64>, sc_smem);
+  if (rc) return rc;
+  if ((rc = set_smem(block_select_kernel<256>, sel_smem))) return rc;
+  const int grp = Hq / Hkv;
+  for (int h0 = 0; h0 < Hq; h0 += chunk) {
+    const int hc = std::min(chunk, Hq - h0);
+    dim3 gs(ntiles, hc);
+    if (d == 128) block_scores_kernel<128><<<gs, 256, sc_smem, st>>>(qbar, kbar, scores, nQB, h0, grp);
+    else block_scores_kernel<64><<<gs, 256, sc_smem, st>>>(qbar, kbar, scores, nQB, h0, grp);
+    if ((rc = launch_check())) return rc;
+    dim3 gsel(nQB, hc);
+    block_select_kernel<256><<<gsel, 256, sel_smem, st>>>(scores, nQB, h0, k_fixed > 0 ? k_fixed : 0, ppm,
+                                                          block_idx, block_cnt, kcap);
+    if ((rc = launch_check())) return rc;
+  }
+  return DSA_OK;
+}
+
+int vertical_slash_index(const void* q, const void* k, int Hq, int Hkv, int n, int d, int last_q, int n_vert,
+                         int n_slash, float scale, int32_t* vert_idx, int32_t* slash_off, int32_t* block_idx,
+                         int32_t* block_cnt, int kcap, int32_t* col_idx, int32_t* col_cnt, int ccap, void* ws,
+                         size_t* ws_bytes, dsa_stream_t stream) {
+  if (!q || !k || !ws_bytes || !block_idx || !block_cnt || !col_idx || !col_cnt) return DSA_ERR_INVALID_ARG;
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n < 64) return DSA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || n % 64 != 0 || last_q != 64 || n > kMaxN) return DSA_ERR_UNSUPPORTED;
+  if ((int64_t)Hq * n >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  if (n_vert < 64 || n_vert > n || n_slash < 1 || n_slash > n) return DSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !aligned16(q) || !aligned16(k)) return DSA_ERR_INVALID_ARG;
+  const int nQB = n / 64;
+  if (kcap < std::min(nQB, 2 * n_slash) || ccap < n_vert) return DSA_ERR_CAPACITY;
+  const int ntiles = nQB;
+  WsCarve c(ws);
+  VSParams p{};
+  p.part = nullptr;
+  uint32_t* status = static_cast<uint32_t*>(c.take(kStatusBytes));
+  (void)status;
+  p.part = static_cast<float*>(c.take((size_t)Hq * ntiles * 64 * 2 * 4));
+  p.lse2 = static_cast<float*>(c.take((size_t)Hq * 64 * 4));
+  p.vert = static_cast<float*>(c.take((size_t)Hq * n * 4));
+  p.slash_part = static_cast<float*>(c.take((size_t)Hq * ntiles * 127 * 4));
+  p.slash = static_cast<float*>(c.take((size_t)Hq * n * 4));
+  p.vsel = vert_idx ? vert_idx : static_cast<int32_t*>(c.take((size_t)Hq * n_vert * 4));
+  p.ssel = slash_off ? slash_off : static_cast<int32_t*>(c.take((size_t)Hq * n_slash * 4));
+  if (!ws) {
+    *ws_bytes = c.off;
+    return DSA_OK;
+  }
+  if (*ws_bytes < c.off) return DSA_ERR_INVALID_ARG;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.block_idx = block_idx;
+  p.block_cnt = block_cnt;
+  p.col_idx = col_idx;
+  p.col_cnt = col_cnt;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.n = n;
+  p.nQB = nQB;
+  p.grp = Hq / Hkv;
+  p.ntiles = ntiles;
+  p.n_vert = n_vert;
+  p.n_slash = n_slash;
+  p.kcap = kcap;
+  p.ccap = ccap;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t smem = (2 * (size_t)d * 64 + 64 * 65) * 4;
+  int rc;
+  dim3 gt(ntiles, Hq);
+  if (d == 128) {
+    if ((rc = set_smem(vs_pass1_kernel<128>, smem)) || (rc = set_smem(vs_pass2_kernel<128>, smem))) return rc;
+    vs_pass1_kernel<128><<<gt, 256, smem, st>>>(p);
+  } else {
+    if ((rc = set_smem(vs_pass1_kernel<64>, smem)) || (rc = set_smem(vs_pass2_kernel<64>, smem))) return rc;
+    vs_pass1_kernel<64><<<gt, 256, smem, st>>>(p);
+  }
+  if ((rc = launch_check())) return rc;
+  vs_lse_kernel<<<Hq, 64, 0, st>>>(p);
+  if ((rc = launch_check())) return rc;
+  if (d == 128) vs_pass2_kernel<128><<<gt, 256, smem, st>>>(p);
+  else vs_pass2_kernel<64><<<gt, 256, smem, st>>>(p);
+  if ((rc = launch_check())) return rc;
+  vs_slash_kernel<<<dim3((n + 255) / 256, Hq), 256, 0, st>>>(p);
+  if ((rc = launch_check())) return rc;
+  vs_topk_kernel<1024><<<dim3(Hq, 2), 1024, 0, st>>>(p);
+  if ((rc = launch_check())) return rc;
+  const size_t plan_smem = (size_t)((nQB + 31) / 32) * 4;
+  if ((rc = set_smem(vs_plan_kernel<256>, plan_smem))) return rc;
+  vs_plan_kernel<256><<<dim3(nQB, Hq), 256, plan_smem, st>>>(p);
+  return launch_check();
+}
+
+int block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, int Hq, int Hkv, int n, int d,
+                          float scale, const int32_t* block_idx, const int32_t* block_cnt, int kcap,
+                          const int32_t* col_idx, const int32_t* col_cnt, int ccap, float* lse, void* ws,
+                          size_t* ws_bytes, dsa_stream_t stream) {
+  if (!q || !k || !v || !o || !block_idx || !block_cnt || !ws_bytes) return DSA_ERR_INVALID_ARG;
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n <= 0 || kcap <= 0) return DSA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || n % 64 != 0 || n > kMaxN) return DSA_ERR_UNSUPPORTED;
+  if ((int64_t)Hq * n >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  if (col_idx && (!col_cnt || ccap <= 0)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!ws) {
+    *ws_bytes = kStatusBytes;
+    return DSA_OK;
+  }
+  if (*ws_bytes < kStatusBytes) return DSA_ERR_INVALID_ARG;
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int nQB = n / 64;
+  if (validate_env()) {
+    validate_lists_kernel<<<dim3(nQB, Hq), 32, 0, st>>>(block_idx, block_cnt, kcap, col_idx, col_cnt, ccap, nQB,
+                                                        Hq, status);
+    if (int rc = launch_check()) return rc;
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, status, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    if (word & kStatusBadList) {
+      cudaMemsetAsync(status, 0, 4, st);
+      cudaStreamSynchronize(st);
+      return DSA_ERR_INVALID_ARG;
+    }
+  }
+  if (d == 128)
+    return launch_attn<128>(q, k, v, o, Hq, Hkv, n, scale, block_idx, block_cnt, kcap, col_idx, col_cnt, ccap, lse,
+                            status, st);
+  return launch_attn<64>(q, k, v, o, Hq, Hkv, n, scale, block_idx, block_cnt, kcap, col_idx, col_cnt, ccap, lse,
+                         status, st);
+}
+
+int sparse_decode_attn(const void* q, const void* k_cache, const void* v_cache, const float* centroids, int B,
+                       int Hq, int Hkv, int S, int d, int keep, int force_last, float scale, void* o,
+                       int32_t* sel_idx, int32_t* sel_cnt, int kcap, void* ws, size_t* ws_bytes,
+                       dsa_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !centroids || !o || !ws_bytes) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S < 64 || keep < 0) return DSA_ERR_INVALID_ARG;
+  if (force_last != 0 && force_last != 1) return DSA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || S % 64 != 0) return DSA_ERR_UNSUPPORTED;
+  {
+    const int gq = Hq / Hkv;
+    if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return DSA_ERR_UNSUPPORTED;
+  }
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(centroids)) return DSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  const int nb = S / 64, grp = Hq / Hkv;
+  const int ncand = force_last ? nb - 1 : nb;
+  const int count = std::min(keep, ncand) + force_last;
+  if (sel_idx && kcap < count) return DSA_ERR_CAPACITY;
+  const size_t sel_smem = (size_t)grp * d * 4 + (size_t)grp * nb * 4 + (size_t)nb * 4 + nb;
+  if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
+  const int nchmax = (nb + kDecChunk - 1) / kDecChunk;
+  WsCarve c(ws);
+  DecodeParams p{};
+  p.status = static_cast<uint32_t*>(c.take(kStatusBytes));
+  p.uidx = static_cast<int32_t*>(c.take((size_t)B * Hkv * nb * 4));
+  p.umask = static_cast<uint8_t*>(c.take((size_t)B * Hkv * nb));
+  p.ucnt = static_cast<int32_t*>(c.take((size_t)B * Hkv * 4));
+  p.part_ml = static_cast<float*>(c.take((size_t)B * Hq * nchmax * 2 * 4));
+  p.part_acc = static_cast<float*>(c.take((size_t)B * Hq * nchmax * d * 4));
+  if (!ws) {
+    *ws_bytes = c.off;
+    return DSA_OK;
+  }
+  if (*ws_bytes < c.off) return DSA_ERR_INVALID_ARG;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kc = static_cast<const __nv_bfloat16*>(k_cache);
+  p.vc = static_cast<const __nv_bfloat16*>(v_cache);
+  p.cent = centroids;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.sel_idx = sel_idx;
+  p.sel_cnt = sel_cnt;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.nb = nb;
+  p.grp = grp;
+  p.keep = keep;
+  p.force_last = force_last;
+  p.kcap = kcap;
+  p.nchmax = nchmax;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int rc;
+  switch (grp * 1000 + d) {
+#define DSA_DECODE_CASE(G, DD)                                                                  \
+  case G * 1000 + DD:                                                                           \
+    rc = launch_decode<DD, G>(p, B, Hkv, nchmax, sel_smem, st);                                 \
+    break;
+    DSA_DECODE_CASE(1, 64) DSA_DECODE_CASE(2, 64) DSA_DECODE_CASE(4, 64) DSA_DECODE_CASE(8, 64)
+    DSA_DECODE_CASE(1, 128) DSA_DECODE_CASE(2, 128) DSA_DECODE_CASE(4, 128) DSA_DECODE_CASE(8, 128)
+#undef DSA_DECODE_CASE
+    default:
+      return DSA_ERR_UNSUPPORTED;
+  }
+  if (rc) return rc;
+  if (d == 128) decode_combine_kernel<128><<<B * Hq, 128, 0, st>>>(p);
+  else decode_combine_kernel<64><<<B * Hq, 128, 0, st>>>(p);
+  return launch_check();
+}
+
+}  // extern "C"

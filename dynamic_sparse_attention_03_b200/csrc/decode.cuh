@@ -1,0 +1,346 @@
+// decode.cuh -- centroid-ranked sparse decode (Squeezed Attention page,
+// "技术方案", online stage: compare the query with every centroid, keep the top
+// clusters, run attention only over the keys and values of those clusters).
+// Clusters are the contiguous 64-token blocks of the cache; centroids are the
+// block means (built by the pooling kernel).
+//
+// Kernels:
+//  decode_select_kernel: one CTA per (batch, KV head): q·c for the GQA group's
+//    q-heads, top `keep` per head (ties to the lower block) plus the last
+//    block, and the union of the group's kept blocks with a per-block head mask.
+//  decode_attn_kernel: one CTA per (batch, KV head, chunk of union blocks).
+//    One producer thread streams whole 64-token K and V blocks (contiguous
+//    16 KB each at d = 128) into a 4-stage shared-memory ring with bulk copies;
+//    4 consumer warps score the block for every q-head that kept it, keep an
+//    online softmax per (warp, head), and merge into one partial per chunk.
+//    Each K/V block is read from HBM once for the whole GQA group.
+//  decode_combine_kernel: merges the chunk partials of each (batch, q-head).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace dsa {
+
+constexpr int kDecChunk = 64;      // union blocks per attention CTA
+constexpr int kDecStages = 4;
+constexpr int kMaxGrp = 8;         // q-heads per KV head supported by the decode path
+
+struct DecodeParams {
+  const __nv_bfloat16* q;      // [B][Hq][D]
+  const __nv_bfloat16* kc;     // [B][Hkv][S][D]
+  const __nv_bfloat16* vc;
+  const float* cent;           // [B][Hkv][nb][D]
+  __nv_bfloat16* o;            // [B][Hq][D]
+  int32_t* sel_idx;            // optional [B][Hq][kcap]
+  int32_t* sel_cnt;            // optional [B][Hq]
+  int32_t* uidx;               // ws [B*Hkv][nb]
+  uint8_t* umask;              // ws [B*Hkv][nb]
+  int32_t* ucnt;               // ws [B*Hkv]
+  float* part_ml;              // ws [B*Hq][nchmax][2]
+  float* part_acc;             // ws [B*Hq][nchmax][D]
+  uint32_t* status;
+  int B, Hq, Hkv, S, nb, grp, keep, force_last, kcap, nchmax;
+  float scale_log2;
+};
+
+// ---------------------------------------------------------------- select
+template <int D, int GRP, int NT>
+__global__ void __launch_bounds__(NT) decode_select_kernel(const DecodeParams p) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  __shared__ SelectSmem sm;
+  const int bg = blockIdx.x;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int nb = p.nb;
+  constexpr int grp = GRP;
+  float* qf = reinterpret_cast<float*>(dsm);                 // [grp][D]
+  float* sc = qf + grp * D;                                   // [grp][nb]
+  int32_t* tmp = reinterpret_cast<int32_t*>(sc + (size_t)grp * nb);   // [nb]
+  uint8_t* mask = reinterpret_cast<uint8_t*>(tmp + nb);      // [nb]
+  for (int x = threadIdx.x; x < grp * D; x += NT) {
+    const int hh = x / D, c = x % D;
+    qf[x] = __bfloat162float(p.q[((size_t)b * p.Hq + g * grp + hh) * D + c]);
+  }
+  for (int x = threadIdx.x; x < nb; x += NT) mask[x] = 0;
+  __syncthreads();
+  // scores: one warp per centroid row, lanes over d
+  constexpr int PER = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float qreg[GRP][PER];
+#pragma unroll
+  for (int hh = 0; hh < grp; ++hh)
+#pragma unroll
+    for (int a = 0; a < PER; ++a) qreg[hh][a] = qf[hh * D + lane * PER + a];
+  const float* crow = p.cent + (size_t)bg * nb * D;
+  for (int t = warp; t < nb; t += NT / 32) {
+    float cv[PER];
+    if (PER == 4) {
+      const float4 v4 = __ldg(reinterpret_cast<const float4*>(crow + (size_t)t * D) + lane);
+      cv[0] = v4.x; cv[1 % PER] = v4.y; cv[2 % PER] = v4.z; cv[3 % PER] = v4.w;
+    } else {
+      const float2 v2 = __ldg(reinterpret_cast<const float2*>(crow + (size_t)t * D) + lane);
+      cv[0] = v2.x; cv[1 % PER] = v2.y;
+    }
+#pragma unroll
+    for (int hh = 0; hh < grp; ++hh) {
+      float s = 0.f;
+#pragma unroll
+      for (int a = 0; a < PER; ++a) s = fmaf(qreg[hh][a], cv[a], s);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+      if (lane == 0) sc[(size_t)hh * nb + t] = s;
+    }
+  }
+  __syncthreads();
+  const int ncand = p.force_last ? nb - 1 : nb;
+  for (int hh = 0; hh < grp; ++hh) {
+    const int cnt = topk_ascending<NT>(sc + (size_t)hh * nb, ncand, p.keep, 0, nb, tmp, nb, sm);
+    __syncthreads();
+    const int h = g * grp + hh;
+    for (int x = threadIdx.x; x < cnt; x += NT) mask[tmp[x]] |= (uint8_t)(1u << hh);
+    if (p.sel_idx) {
+      int32_t* out = p.sel_idx + ((size_t)b * p.Hq + h) * p.kcap;
+      for (int x = threadIdx.x; x < p.kcap; x += NT) out[x] = x < cnt ? tmp[x] : -1;
+    }
+    if (p.sel_cnt && threadIdx.x == 0) p.sel_cnt[(size_t)b * p.Hq + h] = cnt;
+    __syncthreads();
+  }
+  // union of the group's kept blocks, ascending, with head masks
+  const int per = (nb + NT - 1) / NT;
+  const int p0 = min(nb, (int)threadIdx.x * per), p1 = min(nb, p0 + per);
+  int kept = 0;
+  for (int x = p0; x < p1; ++x) kept += mask[x] != 0;
+  int total;
+  int off = block_excl_scan<NT>(kept, sm, total);
+  int32_t* ui = p.uidx + (size_t)bg * nb;
+  uint8_t* um = p.umask + (size_t)bg * nb;
+  for (int x = p0; x < p1; ++x) {
+    if (mask[x]) {
+      ui[off] = x;
+      um[off] = mask[x];
+      ++off;
+    }
+  }
+  if (threadIdx.x == 0) p.ucnt[bg] = total;
+}
+
+// ---------------------------------------------------------------- attention over kept blocks
+template <int D>
+struct DecLayout {
+  static constexpr int kBlkBytes = 64 * D * 2;                  // one 64-token K (or V) block
+  static constexpr int kStage = 2 * kBlkBytes;
+  static constexpr int kRing = kDecStages * kStage;
+  static constexpr int kRed = kRing;                            // warp partials
+  static constexpr int kRedBytes = 4 * kMaxGrp * (D + 2) * 4;
+  static constexpr int kBar = kRed + kRedBytes;
+  static constexpr int kBytes = kBar + 2 * kDecStages * 8 + 16;
+};
+
+template <int D, int GRP>
+__global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams p) {
+  using Lay = DecLayout<D>;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const uint32_t sb = smem_u32(dsm);
+  const int bg = blockIdx.x, chunk = blockIdx.y;
+  const int cnt = p.ucnt[bg];
+  const int u0 = chunk * kDecChunk;
+  if (u0 >= cnt || status_timed_out(p.status)) return;
+  const int u1 = min(cnt, u0 + kDecChunk);
+  const int nu = u1 - u0;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  constexpr int grp = GRP;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar0 = sb + Lay::kBar;
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (kDecStages + s); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + Lay::kBar + 2 * kDecStages * 8);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const AbortState ab{abort_flag, p.status};
+  const int32_t* ui = p.uidx + (size_t)bg * p.nb + u0;
+  const uint8_t* um = p.umask + (size_t)bg * p.nb + u0;
+  const size_t head_base = (size_t)bg * p.S * D;
+
+  if (warp == 4) {
+    // producer: one thread streams whole K and V blocks
+    if (lane == 0) {
+      int u = 0;
+      for (; u < nu; ++u) {
+        const int s = u % kDecStages;
+        if (u >= kDecStages && !mbar_wait(empty(s), ((u / kDecStages) - 1) & 1, ab)) break;
+        const size_t off = head_base + (size_t)ui[u] * 64 * D;
+        mbar_arrive_expect_tx(full(s), 2u * Lay::kBlkBytes);
+        bulk_load(sb + s * Lay::kStage, p.kc + off, Lay::kBlkBytes, full(s));
+        bulk_load(sb + s * Lay::kStage + Lay::kBlkBytes, p.vc + off, Lay::kBlkBytes, full(s));
+      }
+      for (int w = max(0, u - kDecStages); w < u; ++w)
+        mbar_wait_cleanup(full(w % kDecStages), (w / kDecStages) & 1, 200000000ull);
+    }
+    return;
+  }
+  // consumers: warp w takes keys 16w .. 16w+15 of every block; the two half
+  // warps take alternate keys, lane%16 owns dims [8*(lane%16), +8).
+  constexpr int DPL = D / 16;            // dims per lane (8 at d=128, 4 at d=64)
+  const int half = lane >> 4, dl = lane & 15;
+  float qv[GRP][DPL];
+#pragma unroll
+  for (int hh = 0; hh < grp; ++hh)
+#pragma unroll
+    for (int a = 0; a < DPL; ++a)
+      qv[hh][a] = __bfloat162float(p.q[((size_t)b * p.Hq + g * grp + hh) * D + dl * DPL + a]) * p.scale_log2;
+  float m[GRP], l[GRP], acc[GRP][DPL];
+#pragma unroll
+  for (int hh = 0; hh < GRP; ++hh) {
+    m[hh] = -INFINITY;
+    l[hh] = 0.f;
+#pragma unroll
+    for (int a = 0; a < DPL; ++a) acc[hh][a] = 0.f;
+  }
+  bool ok = true;
+  for (int u = 0; u < nu; ++u) {
+    const int s = u % kDecStages;
+    if (!mbar_wait_warp(full(s), (u / kDecStages) & 1, ab)) { ok = false; break; }
+    const uint8_t msk = um[u];
+    const uint8_t* kb = dsm + s * Lay::kStage;
+    const uint8_t* vb = kb + Lay::kBlkBytes;
+    // 8 keys per lane: key = 16*warp + 2*it + half
+    float kf[8][DPL], vf[8][DPL];
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int key = 16 * warp + 2 * it + half;
+      if (DPL == 8) {
+        const uint4 kr = *reinterpret_cast<const uint4*>(kb + key * D * 2 + dl * 16);
+        const uint4 vr = *reinterpret_cast<const uint4*>(vb + key * D * 2 + dl * 16);
+        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const float2 kk = __bfloat1622float2(k2[a]);
+          const float2 vv = __bfloat1622float2(v2[a]);
+          kf[it][(2 * a) % DPL] = kk.x; kf[it][(2 * a + 1) % DPL] = kk.y;
+          vf[it][(2 * a) % DPL] = vv.x; vf[it][(2 * a + 1) % DPL] = vv.y;
+        }
+      } else {
+        const uint2 kr = *reinterpret_cast<const uint2*>(kb + key * D * 2 + dl * 8);
+        const uint2 vr = *reinterpret_cast<const uint2*>(vb + key * D * 2 + dl * 8);
+        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          const float2 kk = __bfloat1622float2(k2[a]);
+          const float2 vv = __bfloat1622float2(v2[a]);
+          kf[it][(2 * a) % DPL] = kk.x; kf[it][(2 * a + 1) % DPL] = kk.y;
+          vf[it][(2 * a) % DPL] = vv.x; vf[it][(2 * a + 1) % DPL] = vv.y;
+        }
+      }
+    }
+    // release the stage once every warp has its registers
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty(s));
+#pragma unroll
+    for (int hh = 0; hh < grp; ++hh) {
+      if (!((msk >> hh) & 1u)) continue;   // block not kept by this head (warp-uniform)
+      float sc[8];
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        float d0 = 0.f;
+#pragma unroll
+        for (int a = 0; a < DPL; ++a) d0 = fmaf(qv[hh][a], kf[it][a], d0);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) d0 += __shfl_xor_sync(0xFFFFFFFFu, d0, o);
+        sc[it] = d0;
+      }
+      float mb = sc[0];
+#pragma unroll
+      for (int it = 1; it < 8; ++it) mb = fmaxf(mb, sc[it]);
+      mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 16));
+      const float mn = fmaxf(m[hh], mb);
+      const float alpha = ex2_approx(m[hh] - mn);   // m = -inf -> 0
+      float ls = 0.f;
+#pragma unroll
+      for (int a = 0; a < DPL; ++a) acc[hh][a] *= alpha;
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const float pe = ex2_approx(sc[it] - mn);
+        ls += pe;
+#pragma unroll
+        for (int a = 0; a < DPL; ++a) acc[hh][a] = fmaf(pe, vf[it][a], acc[hh][a]);
+      }
+      l[hh] = l[hh] * alpha + ls;
+      m[hh] = mn;
+    }
+  }
+  // merge the two half-warps (same dims, same running max), then the 4 warps
+  float* red = reinterpret_cast<float*>(dsm + Lay::kRed);   // [warp][hh][D + 2]
+#pragma unroll
+  for (int hh = 0; hh < grp; ++hh) {
+    l[hh] += __shfl_xor_sync(0xFFFFFFFFu, l[hh], 16);
+#pragma unroll
+    for (int a = 0; a < DPL; ++a) acc[hh][a] += __shfl_xor_sync(0xFFFFFFFFu, acc[hh][a], 16);
+    float* r = red + ((size_t)warp * kMaxGrp + hh) * (D + 2);
+    if (half == 0) {
+#pragma unroll
+      for (int a = 0; a < DPL; ++a) r[dl * DPL + a] = acc[hh][a];
+    }
+    if (lane == 0) {
+      r[D] = m[hh];
+      r[D + 1] = l[hh];
+    }
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (!ok) return;
+  for (int x = threadIdx.x; x < grp * D; x += 128) {
+    const int hh = x / D, c = x % D;
+    float M = -INFINITY;
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, red[((size_t)w * kMaxGrp + hh) * (D + 2) + D]);
+    float a = 0.f, L = 0.f;
+    if (M != -INFINITY) {
+      for (int w = 0; w < 4; ++w) {
+        const float* r = red + ((size_t)w * kMaxGrp + hh) * (D + 2);
+        const float wgt = ex2_approx(r[D] - M);
+        a += wgt * r[c];
+        L += wgt * r[D + 1];
+      }
+    }
+    const size_t ph = (size_t)b * p.Hq + g * grp + hh;
+    p.part_acc[(ph * p.nchmax + chunk) * D + c] = a;
+    if (c == 0) {
+      p.part_ml[(ph * p.nchmax + chunk) * 2 + 0] = M;
+      p.part_ml[(ph * p.nchmax + chunk) * 2 + 1] = L;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- combine
+template <int D>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
+  const int bh = blockIdx.x;   // b*Hq + h
+  const int b = bh / p.Hq, h = bh % p.Hq, g = h / p.grp;
+  const int nch = (p.ucnt[b * p.Hkv + g] + kDecChunk - 1) / kDecChunk;
+  const float* ml = p.part_ml + (size_t)bh * p.nchmax * 2;
+  float M = -INFINITY;
+  for (int c = 0; c < nch; ++c) M = fmaxf(M, ml[2 * c]);
+  for (int x = threadIdx.x; x < D; x += blockDim.x) {
+    float a = 0.f, L = 0.f;
+    if (M != -INFINITY) {
+      for (int c = 0; c < nch; ++c) {
+        const float wgt = ex2_approx(ml[2 * c] - M);
+        a += wgt * p.part_acc[((size_t)bh * p.nchmax + c) * D + x];
+        L += wgt * ml[2 * c + 1];
+      }
+    }
+    p.o[(size_t)bh * D + x] = __float2bfloat16_rn(L > 0.f ? a / L : 0.f);
+  }
+}
+
+}  // namespace dsa
