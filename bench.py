@@ -137,9 +137,15 @@ def max_over_ranks(x: float, world: int) -> float:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(workload: str, rank: int) -> int:
+    """Each rank runs its own independent layer: the workload's seed offset by rank."""
+    return synth.CONFIGS[workload]["seed"] + 1000 * rank
 
 
 def barrier(world: int):
@@ -157,7 +163,7 @@ def run_ours(args, rank, world, local):
     dsa.load_library()
     dev = torch.device("cuda", local)
     p = synth.CONFIGS[args.workload]
-    w = synth.make_prefill(args.workload, device=dev, seed=p["seed"] + 1000 * rank)
+    w = synth.make_prefill(args.workload, device=dev, seed=rank_seed(args.workload, rank))
     Hq, n, d = w.q.shape
     kf, rho = p.get("k_fixed", 0), p.get("keep_ratio", 0.0)
     kcap = dsa.block_index_capacity(n, kf, rho)
