@@ -38,6 +38,7 @@ SYMBOLS = (
     "vertical_slash_index",
     "block_sparse_attn_fwd",
     "sparse_decode_attn",
+    "sparse_decode_attn_static",
     "dsa_get_status",
     "dsa_block_index_capacity",
     "dsa_version",
@@ -71,6 +72,7 @@ _SIGS = {
     "vertical_slash_index": [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _I, _P, _P, _I, _P, _SZ, _P],
     "block_sparse_attn_fwd": [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _I, _P, _P, _I, _P, _P, _SZ, _P],
     "sparse_decode_attn": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P, _SZ, _P],
+    "sparse_decode_attn_static": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P],
     "dsa_get_status": [_P, _P],
     "dsa_block_index_capacity": [_I, _I, _I, _F],
     "dsa_version": [],
@@ -291,4 +293,29 @@ def sparse_decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Te
     args = [_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(centroids), B, Hq, Hkv, S, d, int(keep), int(force_last),
             float(scale), _ptr(o), _ptr(sel_idx), _ptr(sel_cnt), max(kcap, 1)]
     _call_with_ws("sparse_decode_attn", args, q.device, ws)
+    return (o, sel_idx, sel_cnt) if return_sel else o
+
+
+def sparse_decode_attn_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                              centroids: torch.Tensor, keep: int, force_last: int = 1, scale: Optional[float] = None,
+                              return_sel: bool = False, out: Optional[torch.Tensor] = None):
+    """sparse_decode_attn with no workspace: the library's own fixed 32 MiB
+    device array holds the scratch (for callers that cannot allocate device
+    memory).  Calls sharing a device must not overlap on the GPU."""
+    _need_cuda(q, k_cache, v_cache, centroids, out)
+    _need_dtype(centroids, torch.float32, "centroids")
+    B, Hq, d = q.shape
+    Hkv, S = k_cache.shape[1], k_cache.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    nb = S // 64
+    kcap = max(min(keep, nb - 1 if force_last else nb) + (1 if force_last else 0), 1)
+    sel_idx = sel_cnt = None
+    if return_sel:
+        sel_idx = torch.empty((B, Hq, kcap), dtype=torch.int32, device=q.device)
+        sel_cnt = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
+    rc = load_library().sparse_decode_attn_static(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(centroids), B, Hq, Hkv, S, d, int(keep), int(force_last),
+        float(scale), _ptr(o), _ptr(sel_idx), _ptr(sel_cnt), kcap, _stream(q.device))
+    _check(rc, "sparse_decode_attn_static")
     return (o, sel_idx, sel_cnt) if return_sel else o

@@ -18,7 +18,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libdsa.so")
-SOURCES = [os.path.join(HERE, "csrc", "api.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "api.cu"), os.path.join(HERE, "csrc", "decode_static.cu")]
 
 
 def _nvcc() -> str:

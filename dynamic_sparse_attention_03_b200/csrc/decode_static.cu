@@ -1,0 +1,144 @@
+// decode_static.cu -- sparse_decode_attn_static: the centroid-ranked sparse
+// decode of sparse_decode_attn, with its scratch memory in a fixed array that
+// the library itself holds in device memory, for callers that cannot allocate.
+//
+// Who needs it: code that is handed device pointers but has no way to obtain
+// more device memory -- a plugin inside a host application or serving engine
+// whose allocator owns the whole GPU budget and exposes no allocation hook,
+// or a latency-critical decode loop that must never call cudaMalloc (it can
+// synchronize the device and fail under fragmentation).  Such a caller still
+// passes its inputs and outputs, but no workspace.
+//
+// The scratch is one file-scope __device__ array of kStaticScratchBytes
+// (32 MiB); every GPU that loads the library keeps it until the process exits.
+// Host code must not use the array's name as a device address (on the host it
+// names a host-side shadow), so the device address is looked up once per
+// device with cudaGetSymbolAddress, with that device current, and cached.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/dsa.h"
+#include "decode.cuh"
+
+using namespace dsa;
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
+
+std::mutex g_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on the
+// first call per device).  nullptr if the lookup fails.
+void* scratch_on_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
+    g_scratch_addr[dev] = p;
+  }
+  return g_scratch_addr[dev];
+}
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <int D, int G>
+int launch(const DecodeParams& p, int B, int Hkv, int nchmax, size_t sel_smem, cudaStream_t st) {
+  if (sel_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(decode_select_kernel<D, G, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)sel_smem) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  decode_select_kernel<D, G, 256><<<B * Hkv, 256, sel_smem, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaFuncSetAttribute(decode_attn_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           DecLayout<D>::kBytes) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  decode_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 160, DecLayout<D>::kBytes, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  decode_combine_kernel<D><<<B * (Hkv * G), 128, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int sparse_decode_attn_static(const void* q, const void* k_cache, const void* v_cache,
+                                         const float* centroids, int B, int Hq, int Hkv, int S, int d, int keep,
+                                         int force_last, float scale, void* o, int32_t* sel_idx, int32_t* sel_cnt,
+                                         int kcap, dsa_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !centroids || !o) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S < 64 || keep < 0) return DSA_ERR_INVALID_ARG;
+  if (force_last != 0 && force_last != 1) return DSA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || S % 64 != 0) return DSA_ERR_UNSUPPORTED;
+  const int grp = Hq / Hkv;
+  if (grp != 1 && grp != 2 && grp != 4 && grp != 8) return DSA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache) |
+       reinterpret_cast<uintptr_t>(centroids)) & 15u)
+    return DSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  const int nb = S / 64;
+  const int ncand = force_last ? nb - 1 : nb;
+  const int count = (keep < ncand ? keep : ncand) + force_last;
+  if (sel_idx && kcap < count) return DSA_ERR_CAPACITY;
+  const size_t sel_smem = (size_t)grp * d * 4 + (size_t)grp * nb * 4 + (size_t)nb * 4 + nb;
+  if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
+  const int nchmax = (nb + kDecChunk - 1) / kDecChunk;
+  // Scratch layout (same as the workspace of sparse_decode_attn): status word,
+  // union lists and masks, union counts, chunk partials.
+  size_t off = 0;
+  const size_t o_status = off; off = up256(off + 256);
+  const size_t o_uidx = off;   off = up256(off + (size_t)B * Hkv * nb * 4);
+  const size_t o_umask = off;  off = up256(off + (size_t)B * Hkv * nb);
+  const size_t o_ucnt = off;   off = up256(off + (size_t)B * Hkv * 4);
+  const size_t o_ml = off;     off = up256(off + (size_t)B * Hq * nchmax * 2 * 4);
+  const size_t o_acc = off;    off = up256(off + (size_t)B * Hq * nchmax * d * 4);
+  if (off > kStaticScratchBytes) return DSA_ERR_CAPACITY;
+  uint8_t* base = static_cast<uint8_t*>(scratch_on_current_device());
+  if (!base) return DSA_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents: the status word must start at zero.
+  if (cudaMemsetAsync(base + o_status, 0, 256, st) != cudaSuccess) return DSA_ERR_CUDA;
+  DecodeParams p{};
+  p.status = reinterpret_cast<uint32_t*>(base + o_status);
+  p.uidx = reinterpret_cast<int32_t*>(base + o_uidx);
+  p.umask = base + o_umask;
+  p.ucnt = reinterpret_cast<int32_t*>(base + o_ucnt);
+  p.part_ml = reinterpret_cast<float*>(base + o_ml);
+  p.part_acc = reinterpret_cast<float*>(base + o_acc);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kc = static_cast<const __nv_bfloat16*>(k_cache);
+  p.vc = static_cast<const __nv_bfloat16*>(v_cache);
+  p.cent = centroids;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.sel_idx = sel_idx;
+  p.sel_cnt = sel_cnt;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.nb = nb;
+  p.grp = grp;
+  p.keep = keep;
+  p.force_last = force_last;
+  p.kcap = kcap;
+  p.nchmax = nchmax;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  switch (grp * 1000 + d) {
+    case 1064: return launch<64, 1>(p, B, Hkv, nchmax, sel_smem, st);
+    case 2064: return launch<64, 2>(p, B, Hkv, nchmax, sel_smem, st);
+    case 4064: return launch<64, 4>(p, B, Hkv, nchmax, sel_smem, st);
+    case 8064: return launch<64, 8>(p, B, Hkv, nchmax, sel_smem, st);
+    case 1128: return launch<128, 1>(p, B, Hkv, nchmax, sel_smem, st);
+    case 2128: return launch<128, 2>(p, B, Hkv, nchmax, sel_smem, st);
+    case 4128: return launch<128, 4>(p, B, Hkv, nchmax, sel_smem, st);
+    case 8128: return launch<128, 8>(p, B, Hkv, nchmax, sel_smem, st);
+    default: return DSA_ERR_UNSUPPORTED;
+  }
+}

@@ -155,6 +155,34 @@ int sparse_decode_attn(const void* q, const void* k_cache, const void* v_cache, 
                        dsa_stream_t stream);
 
 /*
+ * sparse_decode_attn_static -- sparse_decode_attn without a workspace: the
+ * same computation and arguments (minus ws / ws_bytes), its scratch held in a
+ * fixed 32 MiB array inside the library's device memory.  The pages have no
+ * counterpart of this entry point; it exists for callers that cannot allocate
+ * device memory: a plugin or serving engine whose allocator owns the whole GPU
+ * budget and offers no allocation hook, or a decode loop that must never call
+ * cudaMalloc (it may synchronize the device and can fail once memory is
+ * fragmented).  The caller still passes inputs and outputs.
+ *
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *    Every GPU that loads the library holds the 32 MiB array until exit.
+ *  - Sizes whose scratch exceeds 32 MiB are rejected with DSA_ERR_CAPACITY
+ *    before any launch (e.g. B=16, Hq=32, Hkv=8, S=131072, d=128 needs ~9.9 MB).
+ *  - The first call on a device looks up the array's device address on that
+ *    device (make the device current first); make that first call before any
+ *    stream capture.
+ *  - All calls share the one array, which keeps the previous call's contents;
+ *    each call clears the status word it needs zeroed.  Calls that overlap on
+ *    the GPU (different streams, or other host threads, without ordering
+ *    between them) race on the array.
+ *  - Device-side timeouts are not reported by this entry point (there is no
+ *    workspace to pass to dsa_get_status); launch errors are returned.
+ */
+int sparse_decode_attn_static(const void* q, const void* k_cache, const void* v_cache, const float* centroids,
+                              int B, int Hq, int Hkv, int S, int d, int keep, int force_last, float scale,
+                              void* o, int32_t* sel_idx, int32_t* sel_cnt, int kcap, dsa_stream_t stream);
+
+/*
  * dsa_get_status -- synchronize `stream`, read the workspace's device status
  * word, clear it, and return DSA_OK or the first error recorded on the device
  * (DSA_ERR_TIMEOUT for an expired bounded wait, DSA_ERR_INVALID_ARG for a list
