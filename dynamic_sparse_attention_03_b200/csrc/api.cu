@@ -152,7 +152,7 @@ int launch_attn(const void* q, const void* k, const void* v, void* o, int Hq, in
   int rc = set_smem(bsa_fwd_kernel<D>, smem);
   if (rc) return rc;
   const int64_t grid = (int64_t)Hkv * p.npairs * p.nQB;
-  bsa_fwd_kernel<D><<<(unsigned)grid, 192, smem, st>>>(tq, tk, tv, p);
+  bsa_fwd_kernel<D><<<(unsigned)grid, 224, smem, st>>>(tq, tk, tv, p);
   return launch_check();
 }
 
