@@ -146,13 +146,13 @@ int launch_attn(const void* q, const void* k, const void* v, void* o, int Hq, in
   p.n = n;
   p.nQB = n / 64;
   p.grp = Hq / Hkv;
-  p.npairs = (p.grp + 1) / 2;
+  p.nquads = (p.grp + 3) / 4;
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t smem = AttnLayout<D>::kSmemAlloc;
   int rc = set_smem(bsa_fwd_kernel<D>, smem);
   if (rc) return rc;
-  const int64_t grid = (int64_t)Hkv * p.npairs * p.nQB;
-  bsa_fwd_kernel<D><<<(unsigned)grid, 224, smem, st>>>(tq, tk, tv, p);
+  const int64_t grid = (int64_t)Hkv * p.nquads * p.nQB;
+  bsa_fwd_kernel<D><<<(unsigned)grid, 384, smem, st>>>(tq, tk, tv, p);
   return launch_check();
 }
 

@@ -4,29 +4,34 @@
 // over the key/value blocks the index selected (block-sparse FlashAttention);
 // Fig. 4: slash lines as 64x64 blocks, vertical lines as 1x64 column tiles.
 //
-// Design (one CTA = 7 warps, one work item):
-//  * A work item is 128 query rows that share one KV head: the same 64-token
-//    query block of two q-heads of a GQA group (rows 0-63 = head A, 64-127 =
-//    head B).  Their sorted block lists are merged; each merged entry records
-//    which of the two heads chose it.  Column entries (1x64 tiles) of the two
-//    heads are merged the same way, 64 columns per slot.
-//  * A "tile" is two slots of 64 keys (N = 128 keys).  Warp 0 streams the K
-//    tiles and warp 6 the V tiles, each into its own 3-stage shared-memory ring
-//    (TMA 2D tile loads with 128-byte swizzle for blocks, 16-byte gathers for
-//    columns).  K and V have separate barriers: a K stage is refilled as soon
-//    as its QK^T has run, a V stage once its PV has run, so loads run ahead of
-//    the softmax.  Warp 0 also publishes per-tile metadata (which rows may see
-//    which keys) in a ring with its own barriers.
-//  * Warp 1 (one thread) issues tcgen05.mma: S = Q K^T (M=128, N=128, K=d,
-//    both operands in shared memory) into a double-buffered TMEM S, and
-//    O += P V (M=128, N=d, K=128) with P read from TMEM (double-buffered) and V
-//    from shared memory.  Completion is signalled with tcgen05.commit.
-//  * Warps 2-5 (thread = row = TMEM lane) run the online softmax: tcgen05.ld
-//    of the S row, masks only where a tile needs them, exp2 of
-//    (s*scale*log2e - max) in one FMA, a lazy rescale of O in TMEM only when
-//    the running max grows by more than 2^8, P (bf16) back into TMEM with
-//    tcgen05.st, and the epilogue O / l -> bf16.
-//  * TMEM columns: S0 [0,128) S1 [128,256) O [256,256+d) P0 [384,448) P1 [448,512).
+// Design (one CTA = 12 warps, one work item):
+//  * A work item is one 64-token query block of up to four q-heads that share
+//    a KV head (a GQA group).  Heads 0,1 form the 128-row query tile A, heads
+//    2,3 tile B.  The four sorted block lists are merged; every merged entry
+//    records which heads chose it (a 64-bit key mask per head and slot).
+//    Column entries (1x64 tiles) of the heads are merged the same way, 64
+//    columns per slot.  Each K/V tile therefore crosses shared memory once for
+//    both query tiles.
+//  * A "tile" is two slots of 64 keys (N = 128 keys).  Warp 0 streams K tiles
+//    (and publishes per-tile metadata in a ring with its own barriers), warp 2
+//    streams V tiles, each into a 2-stage ring: TMA 2D tile loads (128-byte
+//    swizzle, no multicast) for blocks, 16-byte gathers for columns.  A K stage
+//    is refilled once both QK^T products have read it, a V stage once both PV
+//    products have.
+//  * Warp 1 (one thread) issues tcgen05.mma in the order QK_A(t+1), PV_B(t),
+//    QK_B(t+1), PV_A(t+1), ...: S = Q K^T (M=128, N=128, K=d, shared-memory
+//    operands) into TMEM S_A / S_B, and O += P V (M=128, N=d, K=128) with P
+//    read from TMEM (aliased onto the first 64 columns of S) and V from shared
+//    memory.  tcgen05.mma operations of a CTA run in issue order, so the PV
+//    that reads P(t) finishes before the next QK^T overwrites S.  While one
+//    softmax warpgroup works on its tile, the tensor pipe runs the other
+//    tile's products.
+//  * Warps 4-7 (tile A) and 8-11 (tile B) run the online softmax, one row per
+//    thread (= TMEM lane): a first pass over the S row for the max, a second
+//    for exp2(s*scale*log2e - max) with packed f32x2 FMAs, P (bf16) written
+//    back into TMEM with tcgen05.st, a lazy rescale of O in TMEM only when the
+//    running max grows by more than 2^8, and the epilogue O / l -> bf16.
+//  * TMEM columns: S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512).
 //  * Every wait is bounded (1 s); on expiry the CTA records a timeout in the
 //    status word, all roles leave their loops, TMEM is freed, the CTA returns.
 #pragma once
@@ -50,20 +55,20 @@ struct AttnParams {
   const int32_t* col_cnt;
   uint32_t* status;
   int kcap, ccap;
-  int Hq, Hkv, n, nQB, grp, npairs;
+  int Hq, Hkv, n, nQB, grp, nquads;
   float scale_log2;
 };
 
-// Per-tile metadata for the MMA issuer and the softmax warps.
+// Per-tile metadata for the MMA issuer and the softmax warpgroups.
 struct alignas(16) AttnMeta {
-  unsigned long long mA[2], mB[2];  // key c of slot s is visible to head A / B rows
-  int blk[2];                       // key block of a block slot, -1 otherwise
-  int kind[2];                      // 0 empty, 1 block, 2 columns
+  unsigned long long m[2][4];  // key c of slot s is visible to the rows of head hh of the item
+  int blk[2];                  // key block of a block slot, -1 otherwise
+  int kind[2];                 // 0 empty, 1 block, 2 columns
   int nslots, last;
 };
 
-constexpr int kAttnKS = 3;   // K stages
-constexpr int kAttnVS = 3;   // V stages
+constexpr int kAttnKS = 2;   // K stages
+constexpr int kAttnVS = 2;   // V stages
 constexpr int kAttnMR = 8;   // metadata ring entries (>= K stages + 2)
 
 template <int D>
@@ -71,8 +76,9 @@ struct AttnLayout {
   static constexpr int NDH = D / 64;              // 64-element (128-byte) column halves of d
   static constexpr int kHalf = 16384;             // one d-half of a 128-row tile (128 x 128 B)
   static constexpr int kTile = NDH * kHalf;       // 128 rows x d bf16
-  static constexpr int kQ = 0;
-  static constexpr int kK0 = kQ + kTile;
+  static constexpr int kQA = 0;
+  static constexpr int kQB = kTile;
+  static constexpr int kK0 = 2 * kTile;
   static constexpr int kV0 = kK0 + kAttnKS * kTile;
   static constexpr int kMeta = kV0 + kAttnVS * kTile;
   static constexpr int kCols = kMeta + kAttnMR * (int)sizeof(AttnMeta);   // [producer][slot][64] ints
@@ -92,7 +98,7 @@ enum : int {
   AB_KEMPTY = AB_KFULL + kAttnKS,
   AB_VFULL = AB_KEMPTY + kAttnKS,
   AB_VEMPTY = AB_VFULL + kAttnVS,
-  AB_SFULL = AB_VEMPTY + kAttnVS,
+  AB_SFULL = AB_VEMPTY + kAttnVS,   // [tile A, tile B]
   AB_PFULL = AB_SFULL + 2,
   AB_PVDONE = AB_PFULL + 2,
   AB_META = AB_PVDONE + 2,
@@ -100,7 +106,7 @@ enum : int {
 };
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256, kTmemP = 384;
+constexpr uint32_t kTmemS = 0, kTmemO = 256;   // + 128 * tile
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, issued by one thread (A from tensor memory).
 __device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
@@ -113,56 +119,81 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, u
       : "memory");
 }
 
-// Merge cursor over the two heads' sorted lists (blocks first, then columns).
+// Merge cursor over the item's heads' sorted lists (blocks first, then columns).
 struct AttnLists {
-  const int32_t *LA, *LB, *CA, *CB;
-  int na, nb, nca, ncb;
+  const int32_t* L[4];
+  const int32_t* C[4];
+  int nl[4], nc[4];
+  int nh;
 };
 
 struct AttnCursor {
-  int ia = 0, ib = 0, ja = 0, jb = 0;
+  int il[4] = {0, 0, 0, 0}, ic[4] = {0, 0, 0, 0};
 
-  __device__ bool more(const AttnLists& L) const { return ia < L.na || ib < L.nb || ja < L.nca || jb < L.ncb; }
+  __device__ bool more_blocks(const AttnLists& A) const {
+    bool r = false;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) r |= (h < A.nh && il[h] < A.nl[h]);
+    return r;
+  }
+  __device__ bool more_cols(const AttnLists& A) const {
+    bool r = false;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) r |= (h < A.nh && ic[h] < A.nc[h]);
+    return r;
+  }
 
   // Forms the next tile (up to two slots of 64 keys) into M; column slots also
   // record their key columns in cols[slot][0..64) (-1 padded).
-  __device__ void next(const AttnLists& L, AttnMeta& M, int (*cols)[64]) {
+  __device__ void next(const AttnLists& A, AttnMeta& M, int (*cols)[64]) {
     for (int sl = 0; sl < 2; ++sl) {
-      if (ia < L.na || ib < L.nb) {
-        const int a = ia < L.na ? L.LA[ia] : 0x7FFFFFFF;
-        const int b = ib < L.nb ? L.LB[ib] : 0x7FFFFFFF;
-        const int blk = min(a, b);
+#pragma unroll
+      for (int h = 0; h < 4; ++h) M.m[sl][h] = 0ull;
+      if (more_blocks(A)) {
+        int v[4];
+        int blk = 0x7FFFFFFF;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          v[h] = (h < A.nh && il[h] < A.nl[h]) ? A.L[h][il[h]] : 0x7FFFFFFF;
+          blk = min(blk, v[h]);
+        }
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+          if (v[h] == blk) {
+            M.m[sl][h] = ~0ull;
+            ++il[h];
+          }
         M.kind[sl] = 1;
         M.blk[sl] = blk;
-        M.mA[sl] = (a == blk) ? ~0ull : 0ull;
-        M.mB[sl] = (b == blk) ? ~0ull : 0ull;
-        ia += (a == blk);
-        ib += (b == blk);
-      } else if (ja < L.nca || jb < L.ncb) {
-        unsigned long long mA = 0, mB = 0;
+      } else if (more_cols(A)) {
         int c = 0;
-        while (c < 64 && (ja < L.nca || jb < L.ncb)) {
-          const int a = ja < L.nca ? L.CA[ja] : 0x7FFFFFFF;
-          const int b = jb < L.ncb ? L.CB[jb] : 0x7FFFFFFF;
-          const int col = min(a, b);
-          if (a == col) { mA |= 1ull << c; ++ja; }
-          if (b == col) { mB |= 1ull << c; ++jb; }
+        while (c < 64 && more_cols(A)) {
+          int v[4];
+          int col = 0x7FFFFFFF;
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            v[h] = (h < A.nh && ic[h] < A.nc[h]) ? A.C[h][ic[h]] : 0x7FFFFFFF;
+            col = min(col, v[h]);
+          }
+#pragma unroll
+          for (int h = 0; h < 4; ++h)
+            if (v[h] == col) {
+              M.m[sl][h] |= 1ull << c;
+              ++ic[h];
+            }
           cols[sl][c] = col;
           ++c;
         }
         for (; c < 64; ++c) cols[sl][c] = -1;
         M.kind[sl] = 2;
         M.blk[sl] = -1;
-        M.mA[sl] = mA;
-        M.mB[sl] = mB;
       } else {
         M.kind[sl] = 0;
         M.blk[sl] = -1;
-        M.mA[sl] = M.mB[sl] = 0ull;
       }
     }
     M.nslots = (M.kind[0] != 0) + (M.kind[1] != 0);
-    M.last = !more(L);
+    M.last = !(more_blocks(A) || more_cols(A));
   }
 };
 
@@ -183,7 +214,7 @@ __device__ __forceinline__ void gather_slot(const __nv_bfloat16* src, const int*
 }
 
 template <int D>
-__global__ void __launch_bounds__(224, 1)
+__global__ void __launch_bounds__(384, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using Lay = AttnLayout<D>;
@@ -201,12 +232,13 @@ __global__ void __launch_bounds__(224, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per_qb = p.Hkv * p.npairs;
+  const int per_qb = p.Hkv * p.nquads;
   const int qb = p.nQB - 1 - (int)(blockIdx.x / per_qb);   // heaviest query blocks first
   const int rem = (int)(blockIdx.x % per_qb);
-  const int g = rem / p.npairs, pr = rem % p.npairs;
-  const int hA = g * p.grp + 2 * pr;
-  const int hB = (2 * pr + 1 < p.grp) ? hA + 1 : -1;
+  const int g = rem / p.nquads, quad = rem % p.nquads;
+  const int h0 = g * p.grp + 4 * quad;
+  const int nh = min(4, p.grp - 4 * quad);
+  const bool hasB = nh > 2;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(AB_Q), 1);
@@ -238,65 +270,71 @@ __global__ void __launch_bounds__(224, 1)
   const uint32_t tmem = *tmem_slot;
   const AbortState ab{abort_flag, p.status};
 
-  const uint32_t sQ = sb + Lay::kQ;
+  auto sQ = [&](int tile) { return sb + (tile ? Lay::kQB : Lay::kQA); };
   auto sK = [&](int s) { return sb + Lay::kK0 + (uint32_t)s * Lay::kTile; };
   auto sV = [&](int s) { return sb + Lay::kV0 + (uint32_t)s * Lay::kTile; };
 
-  AttnLists L;
-  {
-    const size_t rowA = (size_t)hA * p.nQB + qb;
-    const size_t rowB = (size_t)(hB >= 0 ? hB : hA) * p.nQB + qb;
-    L.LA = p.block_idx + rowA * p.kcap;
-    L.LB = p.block_idx + rowB * p.kcap;
-    L.CA = p.col_idx ? p.col_idx + rowA * p.ccap : nullptr;
-    L.CB = p.col_idx ? p.col_idx + rowB * p.ccap : nullptr;
-    L.na = L.nb = L.nca = L.ncb = 0;
-    if (warp == 0 || warp == 6) {
-      L.na = min(max(p.block_cnt[rowA], 0), p.kcap);
-      L.nb = hB >= 0 ? min(max(p.block_cnt[rowB], 0), p.kcap) : 0;
-      L.nca = p.col_idx ? min(max(p.col_cnt[rowA], 0), p.ccap) : 0;
-      L.ncb = (p.col_idx && hB >= 0) ? min(max(p.col_cnt[rowB], 0), p.ccap) : 0;
-    }
-  }
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ K producer + metadata
-    if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      mbar_arrive_expect_tx(bar(AB_Q), (uint32_t)Lay::kTile);
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ producers
+    AttnLists A;
+    A.nh = nh;
 #pragma unroll
-      for (int dh = 0; dh < Lay::NDH; ++dh) {
-        tma_load_2d(sQ + dh * Lay::kHalf, &tmQ, dh * 64, hA * p.n + qb * 64, bar(AB_Q));
-        tma_load_2d(sQ + dh * Lay::kHalf + 8192, &tmQ, dh * 64, (hB >= 0 ? hB : hA) * p.n + qb * 64, bar(AB_Q));
-      }
+    for (int hh = 0; hh < 4; ++hh) {
+      const int h = h0 + min(hh, nh - 1);
+      const size_t row = (size_t)h * p.nQB + qb;
+      A.L[hh] = p.block_idx + row * p.kcap;
+      A.C[hh] = p.col_idx ? p.col_idx + row * p.ccap : nullptr;
+      A.nl[hh] = hh < nh ? min(max(p.block_cnt[row], 0), p.kcap) : 0;
+      A.nc[hh] = (hh < nh && p.col_idx) ? min(max(p.col_cnt[row], 0), p.ccap) : 0;
     }
     AttnCursor cur;
+    const bool isK = (warp == 0);
+    const int NS = isK ? kAttnKS : kAttnVS;
+    if (isK && lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      mbar_arrive_expect_tx(bar(AB_Q), (uint32_t)(2 * Lay::kTile));
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) {
+        const int h = h0 + min(hh, nh - 1);
+#pragma unroll
+        for (int dh = 0; dh < Lay::NDH; ++dh)
+          tma_load_2d(sQ(hh >> 1) + dh * Lay::kHalf + (hh & 1) * 8192, &tmQ, dh * 64, h * p.n + qb * 64, bar(AB_Q));
+      }
+    }
+    if (!isK && lane == 0) prefetch_tmap(&tmV);
+    const CUtensorMap* tm = isK ? &tmK : &tmV;
+    const __nv_bfloat16* base = (isK ? p.k : p.v) + (size_t)g * p.n * D;
+    int(*cols)[64] = isK ? colsK : colsV;
+    const int full0 = isK ? AB_KFULL : AB_VFULL, empty0 = isK ? AB_KEMPTY : AB_VEMPTY;
     int t = 0, issued = 0;
     while (true) {
-      const int ks = t % kAttnKS;
-      if (t >= kAttnKS && !mbar_wait_warp(bar(AB_KEMPTY + ks), ((t / kAttnKS) - 1) & 1, ab)) break;
-      AttnMeta& M = meta[t % kAttnMR];
-      if (lane == 0) cur.next(L, M, colsK);
+      const int s = t % NS;
+      if (t >= NS && !mbar_wait_warp(bar(empty0 + s), ((t / NS) - 1) & 1, ab)) break;
+      AttnMeta& M = isK ? meta[t % kAttnMR] : *vrec;
+      if (lane == 0) cur.next(A, M, cols);
       __syncwarp();
       const int nsl = M.nslots, last = M.last;
+      if (!isK && nsl == 0) break;
       const int k0 = M.kind[0], k1 = M.kind[1];
-      const __nv_bfloat16* kbase = p.k + (size_t)g * p.n * D;
-      if (k0 == 2) gather_slot<D>(kbase, colsK[0], sK(ks), 0, lane);
-      if (k1 == 2) gather_slot<D>(kbase, colsK[1], sK(ks), 1, lane);
+      const int b0 = M.blk[0], b1 = M.blk[1];
+      const uint32_t stg = isK ? sK(s) : sV(s);
+      if (k0 == 2) gather_slot<D>(base, cols[0], stg, 0, lane);
+      if (k1 == 2) gather_slot<D>(base, cols[1], stg, 1, lane);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(bar(AB_META + (t % kAttnMR)));
+        if (isK) mbar_arrive(bar(AB_META + (t % kAttnMR)));
         const uint32_t tx = (uint32_t)((k0 == 1) + (k1 == 1)) * 64u * D * 2u;
-        mbar_arrive_expect_tx(bar(AB_KFULL + ks), tx);
-        for (int sl = 0; sl < 2; ++sl) {
-          if (M.kind[sl] != 1) continue;
-          const int row = g * p.n + M.blk[sl] * 64;
+        mbar_arrive_expect_tx(bar(full0 + s), tx);
+        if (k0 == 1)
 #pragma unroll
           for (int dh = 0; dh < Lay::NDH; ++dh)
-            tma_load_2d(sK(ks) + dh * Lay::kHalf + sl * 8192, &tmK, dh * 64, row, bar(AB_KFULL + ks));
-        }
+            tma_load_2d(stg + dh * Lay::kHalf, tm, dh * 64, g * p.n + b0 * 64, bar(full0 + s));
+        if (k1 == 1)
+#pragma unroll
+          for (int dh = 0; dh < Lay::NDH; ++dh)
+            tma_load_2d(stg + dh * Lay::kHalf + 8192, tm, dh * 64, g * p.n + b1 * 64, bar(full0 + s));
       }
       __syncwarp();
       ++issued;
@@ -304,49 +342,8 @@ __global__ void __launch_bounds__(224, 1)
       ++t;
     }
     if (lane == 0) {
-      for (int u = max(0, issued - kAttnKS); u < issued; ++u)
-        mbar_wait_cleanup(bar(AB_KFULL + (u % kAttnKS)), (u / kAttnKS) & 1, 200000000ull);
-    }
-    __syncwarp();
-  } else if (warp == 6) {
-    // ------------------------------------------------------------ V producer
-    if (lane == 0) prefetch_tmap(&tmV);
-    AttnCursor cur;
-    int t = 0, issued = 0;
-    while (true) {
-      const int vs = t % kAttnVS;
-      if (t >= kAttnVS && !mbar_wait_warp(bar(AB_VEMPTY + vs), ((t / kAttnVS) - 1) & 1, ab)) break;
-      if (lane == 0) cur.next(L, *vrec, colsV);
-      __syncwarp();
-      const int nsl = vrec->nslots, last = vrec->last;
-      if (nsl == 0) break;
-      const int k0 = vrec->kind[0], k1 = vrec->kind[1];
-      const int b0 = vrec->blk[0], b1 = vrec->blk[1];
-      const __nv_bfloat16* vbase = p.v + (size_t)g * p.n * D;
-      if (k0 == 2) gather_slot<D>(vbase, colsV[0], sV(vs), 0, lane);
-      if (k1 == 2) gather_slot<D>(vbase, colsV[1], sV(vs), 1, lane);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        const uint32_t tx = (uint32_t)((k0 == 1) + (k1 == 1)) * 64u * D * 2u;
-        mbar_arrive_expect_tx(bar(AB_VFULL + vs), tx);
-        if (k0 == 1)
-#pragma unroll
-          for (int dh = 0; dh < Lay::NDH; ++dh)
-            tma_load_2d(sV(vs) + dh * Lay::kHalf, &tmV, dh * 64, g * p.n + b0 * 64, bar(AB_VFULL + vs));
-        if (k1 == 1)
-#pragma unroll
-          for (int dh = 0; dh < Lay::NDH; ++dh)
-            tma_load_2d(sV(vs) + dh * Lay::kHalf + 8192, &tmV, dh * 64, g * p.n + b1 * 64, bar(AB_VFULL + vs));
-      }
-      __syncwarp();
-      ++issued;
-      if (last) break;
-      ++t;
-    }
-    if (lane == 0) {
-      for (int u = max(0, issued - kAttnVS); u < issued; ++u)
-        mbar_wait_cleanup(bar(AB_VFULL + (u % kAttnVS)), (u / kAttnVS) & 1, 200000000ull);
+      for (int u = max(0, issued - NS); u < issued; ++u)
+        mbar_wait_cleanup(bar(full0 + (u % NS)), (u / NS) & 1, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -354,115 +351,129 @@ __global__ void __launch_bounds__(224, 1)
     if (lane == 0) {
       const uint32_t idesc_pv = umma_idesc_bf16(128, D, 1);
       bool ok = mbar_wait(bar(AB_Q), 0, ab);
-      int t = 0, prev_nsl = 0;
-      bool have_prev = false;
-      auto issue_pv = [&](int u, int nsl) -> bool {
-        if (!mbar_wait(bar(AB_PFULL + (u & 1)), (u >> 1) & 1, ab)) return false;
-        if (!mbar_wait(bar(AB_VFULL + (u % kAttnVS)), (u / kAttnVS) & 1, ab)) return false;
-        tc_fence_after();
-        const uint32_t vst = sV(u % kAttnVS);
-        const uint32_t pa = tmem + kTmemP + 64u * (uint32_t)(u & 1);
-        for (int kk = 0; kk < nsl * 4; ++kk) {
-          const uint64_t b = umma_desc_sw128(vst + kk * 2048, Lay::kHalf, 1024);
-          umma_bf16_ts(tmem + kTmemO, pa + 8u * (uint32_t)kk, b, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(bar(AB_VEMPTY + (u % kAttnVS)));
-        umma_commit(bar(AB_PVDONE + (u & 1)));
-        return true;
-      };
-      while (ok) {
-        const int ks = t % kAttnKS;
-        if (!mbar_wait(bar(AB_KFULL + ks), (t / kAttnKS) & 1, ab)) { ok = false; break; }
-        const AttnMeta& M = meta[t % kAttnMR];
-        const int nsl = M.nslots;
-        const int last = M.last;
-        if (nsl == 0) break;
-        tc_fence_after();
+      auto qk = [&](int tile, int ks, int nsl) {
         const uint32_t idesc_qk = umma_idesc_bf16(128, nsl * 64, 0);
-        const uint32_t dS = tmem + (uint32_t)(t & 1) * 128u;
+        const uint32_t dS = tmem + kTmemS + 128u * (uint32_t)tile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = umma_desc_sw128(sQ + (kk >> 2) * Lay::kHalf + (kk & 3) * 32, 16, 1024);
+          const uint64_t a = umma_desc_sw128(sQ(tile) + (kk >> 2) * Lay::kHalf + (kk & 3) * 32, 16, 1024);
           const uint64_t b = umma_desc_sw128(sK(ks) + (kk >> 2) * Lay::kHalf + (kk & 3) * 32, 16, 1024);
           umma_bf16_ss(dS, a, b, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar(AB_SFULL + (t & 1)));
-        umma_commit(bar(AB_KEMPTY + ks));
-        if (have_prev && !issue_pv(t - 1, prev_nsl)) { ok = false; break; }
-        prev_nsl = nsl;
-        have_prev = true;
+        umma_commit(bar(AB_SFULL + tile));
+      };
+      auto pv = [&](int tile, int u, int nsl) {
+        const uint32_t vst = sV(u % kAttnVS);
+        const uint32_t pa = tmem + kTmemS + 128u * (uint32_t)tile;   // P aliases the first 64 columns of S
+        for (int kk = 0; kk < nsl * 4; ++kk) {
+          const uint64_t b = umma_desc_sw128(vst + kk * 2048, Lay::kHalf, 1024);
+          umma_bf16_ts(tmem + kTmemO + 128u * (uint32_t)tile, pa + 8u * (uint32_t)kk, b, idesc_pv,
+                       (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar(AB_PVDONE + tile));
+      };
+      int t = 0;
+      int nsl = 0, last = 1;
+      if (ok) ok = mbar_wait(bar(AB_KFULL), 0, ab);
+      if (ok) {
+        nsl = meta[0].nslots;
+        last = meta[0].last;
+        if (nsl > 0) {
+          tc_fence_after();
+          qk(0, 0, nsl);
+          if (hasB) qk(1, 0, nsl);
+          umma_commit(bar(AB_KEMPTY));
+        }
+      }
+      while (ok && nsl > 0) {
+        int nsl_next = 0, last_next = 1;
+        // PV_A(t) ; QK_A(t+1)
+        if (!mbar_wait(bar(AB_PFULL + 0), t & 1, ab)) { ok = false; break; }
+        if (!mbar_wait(bar(AB_VFULL + (t % kAttnVS)), (t / kAttnVS) & 1, ab)) { ok = false; break; }
+        tc_fence_after();
+        pv(0, t, nsl);
+        if (!last) {
+          const int ks = (t + 1) % kAttnKS;
+          if (!mbar_wait(bar(AB_KFULL + ks), ((t + 1) / kAttnKS) & 1, ab)) { ok = false; break; }
+          nsl_next = meta[(t + 1) % kAttnMR].nslots;
+          last_next = meta[(t + 1) % kAttnMR].last;
+          tc_fence_after();
+          qk(0, ks, nsl_next);
+        }
+        // PV_B(t) ; QK_B(t+1)
+        if (hasB) {
+          if (!mbar_wait(bar(AB_PFULL + 1), t & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          pv(1, t, nsl);
+          if (!last) qk(1, (t + 1) % kAttnKS, nsl_next);
+        }
+        umma_commit(bar(AB_VEMPTY + (t % kAttnVS)));
+        if (!last) umma_commit(bar(AB_KEMPTY + ((t + 1) % kAttnKS)));
         if (last) break;
+        nsl = nsl_next;
+        last = last_next;
         ++t;
       }
-      if (ok && have_prev) issue_pv(t, prev_nsl);
       // Drain: every MMA of this CTA has completed before TMEM is freed.
       umma_commit(bar(AB_DRAIN));
       mbar_wait_cleanup(bar(AB_DRAIN), 0, 200000000ull);
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ softmax / epilogue (warps 2-5)
-    const int q4 = warp & 3;
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int tile = (warp - 4) >> 2;     // 0: warps 4-7, 1: warps 8-11
+    const int q4 = warp & 3;              // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;
-    const int grpB = row >> 6;
+    const int hh = 2 * tile + (row >> 6);  // head of the item for this row
     const int r = row & 63;
+    const bool active = (tile == 0) || hasB;
     const uint32_t laddr = tmem + ((uint32_t)(q4 * 32) << 16);
+    const uint32_t sS = laddr + kTmemS + 128u * (uint32_t)tile;
+    const uint32_t sO = laddr + kTmemO + 128u * (uint32_t)tile;
     const unsigned long long causal = (r == 63) ? ~0ull : ((1ull << (r + 1)) - 1ull);
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     int t = 0;
     bool ok = true, any = false;
-    while (true) {
+    while (active) {
       if (!mbar_wait_warp(bar(AB_META + (t % kAttnMR)), (t / kAttnMR) & 1, ab)) { ok = false; break; }
       const AttnMeta& M = meta[t % kAttnMR];
       const int nsl = M.nslots;
       if (nsl == 0) break;
       const int last = M.last;
-      unsigned long long vm0 = grpB ? M.mB[0] : M.mA[0];
+      unsigned long long vm0 = M.m[0][hh];
       if (M.kind[0] == 1 && M.blk[0] == qb) vm0 &= causal;
       unsigned long long vm1 = 0ull;
       if (nsl > 1) {
-        vm1 = grpB ? M.mB[1] : M.mA[1];
+        vm1 = M.m[1][hh];
         if (M.kind[1] == 1 && M.blk[1] == qb) vm1 &= causal;
       }
-      if (!mbar_wait_warp(bar(AB_SFULL + (t & 1)), (t >> 1) & 1, ab)) { ok = false; break; }
+      const bool masked = __any_sync(0xFFFFFFFFu, (vm0 & vm1) != ~0ull);
+      if (!mbar_wait_warp(bar(AB_SFULL + tile), t & 1, ab)) { ok = false; break; }
       tc_fence_after();
-      uint32_t r0[32], r1[32], r2[32], r3[32];
-      const uint32_t sa = laddr + (uint32_t)(t & 1) * 128u;
-      tmem_ld32(sa, r0);
-      tmem_ld32(sa + 32, r1);
-      tmem_ld32(sa + 64, r2);
-      tmem_ld32(sa + 96, r3);
-      tmem_wait_ld();
-      reg_fence(r0);
-      reg_fence(r1);
-      reg_fence(r2);
-      reg_fence(r3);
-      float x[128];
+      // pass 1: row max of the raw scores (the scale is positive, so it commutes)
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        x[c] = __uint_as_float(r0[c]);
-        x[32 + c] = __uint_as_float(r1[c]);
-        x[64 + c] = __uint_as_float(r2[c]);
-        x[96 + c] = __uint_as_float(r3[c]);
-      }
-      if (__any_sync(0xFFFFFFFFu, (vm0 & vm1) != ~0ull)) {
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(sS + 64 * h2, ra);
+        tmem_ld32(sS + 64 * h2 + 32, rb);
+        tmem_wait_ld();
+        reg_fence(ra);
+        reg_fence(rb);
+        const unsigned long long vm = h2 ? vm1 : vm0;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = ((vm0 >> c) & 1ull) ? x[c] : -INFINITY;
-          x[64 + c] = ((vm1 >> c) & 1ull) ? x[64 + c] : -INFINITY;
+        for (int c = 0; c < 32; ++c) {
+          float a = __uint_as_float(ra[c]), b = __uint_as_float(rb[c]);
+          if (masked) {
+            a = ((vm >> c) & 1ull) ? a : -INFINITY;
+            b = ((vm >> (32 + c)) & 1ull) ? b : -INFINITY;
+          }
+          mx0 = fmaxf(mx0, a);
+          mx1 = fmaxf(mx1, b);
         }
       }
-      // row max of the raw scores (the scale is positive, so it commutes)
-      float mt0 = x[0], mt1 = x[1], mt2 = x[2], mt3 = x[3];
-#pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mt0 = fmaxf(mt0, x[c]);
-        mt1 = fmaxf(mt1, x[c + 1]);
-        mt2 = fmaxf(mt2, x[c + 2]);
-        mt3 = fmaxf(mt3, x[c + 3]);
-      }
-      const float mt = fmaxf(fmaxf(mt0, mt1), fmaxf(mt2, mt3)) * sl2;
+      const float mt = fmaxf(mx0, mx1) * sl2;
       float m_new = m_run;
       bool rescale = false;
       if (m_run == -INFINITY) {
@@ -473,62 +484,67 @@ __global__ void __launch_bounds__(224, 1)
       }
       const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
       const float nmu = (m_new == -INFINITY) ? 0.f : -m_new;
-      // p = 2^(s*scale*log2e - m): two lanes per packed FMA
-      float2 s01 = make_float2(0.f, 0.f), s23 = s01;
+      // pass 2: p = 2^(s*scale*log2e - m), P (bf16, two keys per column) over
+      // the first 64 columns of S: chunk 2*h2 and 2*h2+1 are read before the
+      // 32 columns at 32*h2 are written, and those columns were read earlier.
+      float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        const float2 a = ffma2(make_float2(x[c], x[c + 1]), make_float2(sl2, sl2), make_float2(nmu, nmu));
-        const float2 b = ffma2(make_float2(x[c + 2], x[c + 3]), make_float2(sl2, sl2), make_float2(nmu, nmu));
-        x[c] = ex2_approx(a.x);
-        x[c + 1] = ex2_approx(a.y);
-        x[c + 2] = ex2_approx(b.x);
-        x[c + 3] = ex2_approx(b.y);
-        s01 = fadd2(s01, make_float2(x[c], x[c + 1]));
-        s23 = fadd2(s23, make_float2(x[c + 2], x[c + 3]));
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(sS + 64 * h2, ra);
+        tmem_ld32(sS + 64 * h2 + 32, rb);
+        tmem_wait_ld();
+        reg_fence(ra);
+        reg_fence(rb);
+        const unsigned long long vm = h2 ? vm1 : vm0;
+        uint32_t pk[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float a0 = __uint_as_float(ra[2 * j]), a1 = __uint_as_float(ra[2 * j + 1]);
+          float b0 = __uint_as_float(rb[2 * j]), b1 = __uint_as_float(rb[2 * j + 1]);
+          if (masked) {
+            a0 = ((vm >> (2 * j)) & 1ull) ? a0 : -INFINITY;
+            a1 = ((vm >> (2 * j + 1)) & 1ull) ? a1 : -INFINITY;
+            b0 = ((vm >> (32 + 2 * j)) & 1ull) ? b0 : -INFINITY;
+            b1 = ((vm >> (33 + 2 * j)) & 1ull) ? b1 : -INFINITY;
+          }
+          const float2 ea = ffma2(make_float2(a0, a1), make_float2(sl2, sl2), make_float2(nmu, nmu));
+          const float2 eb = ffma2(make_float2(b0, b1), make_float2(sl2, sl2), make_float2(nmu, nmu));
+          const float2 pa = make_float2(ex2_approx(ea.x), ex2_approx(ea.y));
+          const float2 pb = make_float2(ex2_approx(eb.x), ex2_approx(eb.y));
+          sum2 = fadd2(sum2, fadd2(pa, pb));
+          pk[j] = pack_bf16x2(pa.x, pa.y);
+          pk[16 + j] = pack_bf16x2(pb.x, pb.y);
+        }
+        tmem_st32(sS + 32 * h2, pk);
       }
-      l_run = l_run * alpha + ((s01.x + s01.y) + (s23.x + s23.y));
+      l_run = l_run * alpha + (sum2.x + sum2.y);
       m_run = m_new;
-      // P buffer t&1 was read by PV(t-2); a rescale of O needs PV(t-1) done.
-      const bool any_rescale = __any_sync(0xFFFFFFFFu, rescale);
-      if (any_rescale && t >= 1) {
-        if (!mbar_wait_warp(bar(AB_PVDONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ab)) { ok = false; break; }
-      } else if (t >= 2) {
-        if (!mbar_wait_warp(bar(AB_PVDONE + (t & 1)), ((t - 2) >> 1) & 1, ab)) { ok = false; break; }
-      }
-      tc_fence_after();
-      if (any_rescale && t >= 1) {
+      // O rescale: the PV of the previous tile has completed (it was issued
+      // before this tile's QK^T, and the tensor pipe runs in order).
+      if (__any_sync(0xFFFFFFFFu, rescale)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
-          tmem_ld32(laddr + kTmemO + c * 32, ov);
+          tmem_ld32(sO + c * 32, ov);
           tmem_wait_ld();
           reg_fence(ov);
 #pragma unroll
           for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-          tmem_st32(laddr + kTmemO + c * 32, ov);
+          tmem_st32(sO + c * 32, ov);
         }
-      }
-      // P (bf16, two keys per 32-bit column) into TMEM buffer t&1: the A operand of PV.
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(x[2 * j], x[2 * j + 1]);
-        tmem_st32(laddr + kTmemP + 64u * (uint32_t)(t & 1), pk);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(x[64 + 2 * j], x[64 + 2 * j + 1]);
-        tmem_st32(laddr + kTmemP + 64u * (uint32_t)(t & 1) + 32u, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(AB_PFULL + (t & 1)));
+      mbar_arrive(bar(AB_PFULL + tile));
       any = true;
       if (last) break;
       ++t;
     }
-    if (ok && any) ok = mbar_wait_warp(bar(AB_PVDONE + (t & 1)), (t >> 1) & 1, ab);
-    const int h = grpB ? hB : hA;
-    if (ok && h >= 0) {
+    if (active && ok && any) ok = mbar_wait_warp(bar(AB_PVDONE + tile), t & 1, ab);
+    if (active && ok && hh < nh) {
       tc_fence_after();
+      const int h = h0 + hh;
       const int i = qb * 64 + r;
       const float inv = (any && l_run > 0.f) ? 1.0f / l_run : 0.f;
       __nv_bfloat16* orow = p.o + ((size_t)h * p.n + i) * D;
@@ -536,7 +552,7 @@ __global__ void __launch_bounds__(224, 1)
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
         if (any) {
-          tmem_ld32(laddr + kTmemO + c * 32, ov);
+          tmem_ld32(sO + c * 32, ov);
           tmem_wait_ld();
           reg_fence(ov);
         } else {
