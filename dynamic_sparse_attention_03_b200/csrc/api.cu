@@ -239,23 +239,34 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   if (d == 128) pool_blocks_kernel<128><<<(unsigned)((int64_t)Hq * nQB), 256, 0, st>>>(qp, qbar, (int64_t)Hq * nQB);
   else pool_blocks_kernel<64><<<(unsigned)((int64_t)Hq * nQB), 256, 0, st>>>(qp, qbar, (int64_t)Hq * nQB);
   if (int rc = launch_check()) return rc;
-  const int ntr = (nQB + 63) / 64;
+  const int ntr = (nQB + kScoreTile - 1) / kScoreTile;
   const unsigned ntiles = (unsigned)(ntr * (ntr + 1) / 2);
-  const size_t sc_smem = 2 * (size_t)d * 64 * 4;
-  const size_t sel_smem = (size_t)nQB * 4;
-  int rc = (d == 128) ? set_smem(block_scores_kernel<128>, sc_smem) : set_smem(block_scores_kernel<64>, sc_smem);
+  constexpr int kSelWarps = 4;
+  const bool warp_select = nQB <= 4096;   // a row per warp in shared memory
+  const size_t sel_smem = warp_select ? (size_t)kSelWarps * nQB * 4 : (size_t)nQB * 4;
+  int rc = (d == 128) ? set_smem(block_scores_kernel<128>, kScoreSmem) : set_smem(block_scores_kernel<64>, kScoreSmem);
   if (rc) return rc;
-  if ((rc = set_smem(block_select_kernel<256>, sel_smem))) return rc;
+  if (warp_select) {
+    if ((rc = set_smem(block_select_warp_kernel<kSelWarps>, sel_smem))) return rc;
+  } else if ((rc = set_smem(block_select_kernel<256>, sel_smem))) {
+    return rc;
+  }
   const int grp = Hq / Hkv;
+  const int kf = k_fixed > 0 ? k_fixed : 0;
   for (int h0 = 0; h0 < Hq; h0 += chunk) {
     const int hc = std::min(chunk, Hq - h0);
     dim3 gs(ntiles, hc);
-    if (d == 128) block_scores_kernel<128><<<gs, 256, sc_smem, st>>>(qbar, kbar, scores, nQB, h0, grp);
-    else block_scores_kernel<64><<<gs, 256, sc_smem, st>>>(qbar, kbar, scores, nQB, h0, grp);
+    if (d == 128) block_scores_kernel<128><<<gs, 256, kScoreSmem, st>>>(qbar, kbar, scores, nQB, h0, grp);
+    else block_scores_kernel<64><<<gs, 256, kScoreSmem, st>>>(qbar, kbar, scores, nQB, h0, grp);
     if ((rc = launch_check())) return rc;
-    dim3 gsel(nQB, hc);
-    block_select_kernel<256><<<gsel, 256, sel_smem, st>>>(scores, nQB, h0, k_fixed > 0 ? k_fixed : 0, ppm,
-                                                          block_idx, block_cnt, kcap);
+    if (warp_select) {
+      const int nrows = hc * nQB;
+      block_select_warp_kernel<kSelWarps><<<(nrows + kSelWarps - 1) / kSelWarps, kSelWarps * 32, sel_smem, st>>>(
+          scores, nQB, h0, nrows, kf, ppm, block_idx, block_cnt, kcap);
+    } else {
+      block_select_kernel<256><<<dim3(nQB, hc), 256, sel_smem, st>>>(scores, nQB, h0, kf, ppm, block_idx, block_cnt,
+                                                                     kcap);
+    }
     if ((rc = launch_check())) return rc;
   }
   return DSA_OK;
