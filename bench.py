@@ -1,7 +1,7 @@
 """Benchmark of the dynamic-sparse-attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-decode] [--no-e2e] [--no-cpu-baseline]
+                    [--workload NAME] [--no-decode] [--no-vs] [--no-e2e] [--no-cpu-baseline]
 
 A step is one prefill layer of the block-sparse path on the named workload
 (default: the LLaMA-3-8B-shaped layer at 128K tokens, 32 q-heads / 8 KV
@@ -217,6 +217,19 @@ def run_ours(args, rank, world, local):
     achieved = flops / (attn_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     density = float(bc.to(torch.float64).sum().item()) / (Hq * (n // 64) * (n // 64 + 1) / 2)
+    # index estimation: algorithmic bytes = Q and K read once (bf16); FLOPs = the
+    # pooled scores of every causal (query block, key block) pair, fp32 FMA.
+    nqb = n // 64
+    idx_bytes = (Hq + w.k.shape[0]) * n * d * 2
+    idx_flops = 2.0 * d * Hq * nqb * (nqb + 1) / 2
+    fp32_peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
+    index_roof = {"kernels": "pool_blocks + block_scores + block_select",
+                  "hbm": {"achieved": round(idx_bytes / (index_ms * 1e-3) / 1e9, 1), "peak": peaks["hbm_gbs"],
+                          "unit": "GB/s", "frac": round(idx_bytes / (index_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                          "bytes": idx_bytes},
+                  "alu": {"achieved": round(idx_flops / (index_ms * 1e-3) / 1e12, 2), "peak": round(fp32_peak, 1),
+                          "unit": "TFLOP/s fp32", "frac": round(idx_flops / (index_ms * 1e-3) / 1e12 / fp32_peak, 4),
+                          "flops": idx_flops, "peak_source": "148 SMs x 128 FMA/clk x 2 x max SM clock"}}
     res = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
@@ -227,6 +240,7 @@ def run_ours(args, rank, world, local):
                    "l2": "inputs larger than L2 (Q 1.07 GB, K/V 268 MB each at 128K), no flush",
                    "parallelism": f"independent layer per GPU x{world}"},
         "breakdown_ms": {"index": round(index_ms, 4), "attention": round(attn_ms, 4)},
+        "index_roofline": index_roof,
         "effective_flops_per_step": flops,
         "roofline": {"bound": "tensor", "kernel": "bsa_fwd_kernel<128>", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
@@ -292,6 +306,51 @@ def run_decode(args, local):
             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": total,
             "union_kv_blocks": union_blocks, "centroid_build_ms": round(cent_ms, 4),
             "centroid_build_GB/s": round(cent_gbs, 1), "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": src}
+
+
+def run_vs(args, local):
+    """Vertical-slash prefill layer at 128K: vertical_slash_index followed by
+    block_sparse_attn_fwd over the plan's blocks and column tiles.  Effective
+    FLOPs count the selected blocks (the diagonal block at its causal elements)
+    plus 4*d FLOP per (row, kept column) pair of every column tile entry."""
+    import dynamic_sparse_attention_03_b200 as dsa
+
+    dev = torch.device("cuda", local)
+    name = "llama3-8b-128k-vs"
+    p = synth.CONFIGS[name]
+    w = synth.make_prefill(name, device=dev)
+    Hq, n, d = w.q.shape
+    ws = dsa.Workspace(dev)
+    res = dsa.vertical_slash_index(w.q, w.k, p["n_vert"], p["n_slash"], ws=ws)
+    o = dsa.block_sparse_attn_fwd(w.q, w.k, w.v, res["block_idx"], res["block_cnt"], res["col_idx"],
+                                  res["col_cnt"], ws=ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    reps = 2
+    ev[0].record(stream)
+    for _ in range(reps):
+        dsa.vertical_slash_index(w.q, w.k, p["n_vert"], p["n_slash"], ws=ws)
+    ev[1].record(stream)
+    for _ in range(reps):
+        dsa.block_sparse_attn_fwd(w.q, w.k, w.v, res["block_idx"], res["block_cnt"], res["col_idx"],
+                                  res["col_cnt"], out=o, ws=ws)
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    idx_ms = ev[0].elapsed_time(ev[1]) / reps
+    att_ms = ev[1].elapsed_time(ev[2]) / reps
+    flops = prefill_flops(res["block_cnt"], d) + float(res["col_cnt"].to(torch.float64).sum().item()) * 4 * d * 64
+    nqb = n // 64
+    density = float(res["block_cnt"].to(torch.float64).sum().item()) / (Hq * nqb * (nqb + 1) / 2)
+    peaks, _ = load_peaks()
+    tf = flops / (att_ms * 1e-3) / 1e12
+    out = {"workload": name, "index_ms": round(idx_ms, 3), "attention_ms": round(att_ms, 3),
+           "ms_per_layer": round(idx_ms + att_ms, 3), "effective_tflops_attention": round(tf, 1),
+           "frac_attention": round(tf / peaks.get("bf16_tflops_sustained", 1362.1), 4),
+           "selected_block_density": round(density, 4), "status": dsa.get_status(ws)}
+    del w, res, o
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, ctx, local):
@@ -407,6 +466,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama3-8b-128k-bs10")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-vs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -425,6 +485,8 @@ def main():
         res["e2e"] = run_e2e(args, ctx, local)
     if not args.no_decode:
         res["decode"] = run_decode(args, local)
+    if not args.no_vs:
+        res["vertical_slash"] = run_vs(args, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, secs, cores = oracle_sample(args.workload, 15.0, w=ctx[0])
         res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,

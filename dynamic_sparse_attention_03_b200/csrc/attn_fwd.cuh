@@ -448,32 +448,50 @@ __global__ void __launch_bounds__(384, 1)
         vm1 = M.m[1][hh];
         if (M.kind[1] == 1 && M.blk[1] == qb) vm1 &= causal;
       }
-      const bool masked = __any_sync(0xFFFFFFFFu, (vm0 & vm1) != ~0ull);
+      // Per slot and row: every key visible, none visible, or a partial mask
+      // (the diagonal block, column slots).  Warps whose rows are all "every" or
+      // "none" take the fast path: a hidden slot gets FMA scale 0 and bias
+      // -inf, so its exp2 is 0 without any per-key work.
+      const bool none0 = vm0 == 0ull, none1 = vm1 == 0ull;
+      const bool fast0 = __all_sync(0xFFFFFFFFu, none0 || vm0 == ~0ull);
+      const bool fast1 = __all_sync(0xFFFFFFFFu, none1 || vm1 == ~0ull);
       if (!mbar_wait_warp(bar(AB_SFULL + tile), t & 1, ab)) { ok = false; break; }
       tc_fence_after();
       // pass 1: row max of the raw scores (the scale is positive, so it commutes)
-      float mx0 = -INFINITY, mx1 = -INFINITY;
+      float mx = -INFINITY;
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int sl = 0; sl < 2; ++sl) {
+        if (sl >= nsl) break;
         uint32_t ra[32], rb[32];
-        tmem_ld32(sS + 64 * h2, ra);
-        tmem_ld32(sS + 64 * h2 + 32, rb);
+        tmem_ld32(sS + 64 * sl, ra);
+        tmem_ld32(sS + 64 * sl + 32, rb);
         tmem_wait_ld();
         reg_fence(ra);
         reg_fence(rb);
-        const unsigned long long vm = h2 ? vm1 : vm0;
+        const unsigned long long vm = sl ? vm1 : vm0;
+        float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
+        if (sl ? fast1 : fast0) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          float a = __uint_as_float(ra[c]), b = __uint_as_float(rb[c]);
-          if (masked) {
-            a = ((vm >> c) & 1ull) ? a : -INFINITY;
-            b = ((vm >> (32 + c)) & 1ull) ? b : -INFINITY;
+          for (int c = 0; c < 32; c += 2) {
+            c0 = fmaxf(c0, __uint_as_float(ra[c]));
+            c1 = fmaxf(c1, __uint_as_float(ra[c + 1]));
+            c2 = fmaxf(c2, __uint_as_float(rb[c]));
+            c3 = fmaxf(c3, __uint_as_float(rb[c + 1]));
           }
-          mx0 = fmaxf(mx0, a);
-          mx1 = fmaxf(mx1, b);
+          if (sl ? none1 : none0) c0 = c1 = c2 = c3 = -INFINITY;
+        } else {
+          const uint32_t lo = (uint32_t)vm, hi = (uint32_t)(vm >> 32);
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            c0 = fmaxf(c0, ((lo >> c) & 1u) ? __uint_as_float(ra[c]) : -INFINITY);
+            c1 = fmaxf(c1, ((lo >> (c + 1)) & 1u) ? __uint_as_float(ra[c + 1]) : -INFINITY);
+            c2 = fmaxf(c2, ((hi >> c) & 1u) ? __uint_as_float(rb[c]) : -INFINITY);
+            c3 = fmaxf(c3, ((hi >> (c + 1)) & 1u) ? __uint_as_float(rb[c + 1]) : -INFINITY);
+          }
         }
+        mx = fmaxf(mx, fmaxf(fmaxf(c0, c1), fmaxf(c2, c3)));
       }
-      const float mt = fmaxf(mx0, mx1) * sl2;
+      const float mt = mx * sl2;
       float m_new = m_run;
       bool rescale = false;
       if (m_run == -INFINITY) {
@@ -489,34 +507,50 @@ __global__ void __launch_bounds__(384, 1)
       // 32 columns at 32*h2 are written, and those columns were read earlier.
       float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int sl = 0; sl < 2; ++sl) {
+        if (sl >= nsl) break;
         uint32_t ra[32], rb[32];
-        tmem_ld32(sS + 64 * h2, ra);
-        tmem_ld32(sS + 64 * h2 + 32, rb);
+        tmem_ld32(sS + 64 * sl, ra);
+        tmem_ld32(sS + 64 * sl + 32, rb);
         tmem_wait_ld();
         reg_fence(ra);
         reg_fence(rb);
-        const unsigned long long vm = h2 ? vm1 : vm0;
+        const bool none = sl ? none1 : none0;
+        const float k2 = none ? 0.f : sl2;             // hidden slot: 2^(0*s - inf) = 0
+        const float b2 = none ? -INFINITY : nmu;
         uint32_t pk[32];
+        if (sl ? fast1 : fast0) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float a0 = __uint_as_float(ra[2 * j]), a1 = __uint_as_float(ra[2 * j + 1]);
-          float b0 = __uint_as_float(rb[2 * j]), b1 = __uint_as_float(rb[2 * j + 1]);
-          if (masked) {
-            a0 = ((vm >> (2 * j)) & 1ull) ? a0 : -INFINITY;
-            a1 = ((vm >> (2 * j + 1)) & 1ull) ? a1 : -INFINITY;
-            b0 = ((vm >> (32 + 2 * j)) & 1ull) ? b0 : -INFINITY;
-            b1 = ((vm >> (33 + 2 * j)) & 1ull) ? b1 : -INFINITY;
+          for (int j = 0; j < 16; ++j) {
+            const float2 ea = ffma2(make_float2(__uint_as_float(ra[2 * j]), __uint_as_float(ra[2 * j + 1])),
+                                    make_float2(k2, k2), make_float2(b2, b2));
+            const float2 eb = ffma2(make_float2(__uint_as_float(rb[2 * j]), __uint_as_float(rb[2 * j + 1])),
+                                    make_float2(k2, k2), make_float2(b2, b2));
+            const float2 pa = make_float2(ex2_approx(ea.x), ex2_approx(ea.y));
+            const float2 pb = make_float2(ex2_approx(eb.x), ex2_approx(eb.y));
+            sum2 = fadd2(sum2, fadd2(pa, pb));
+            pk[j] = pack_bf16x2(pa.x, pa.y);
+            pk[16 + j] = pack_bf16x2(pb.x, pb.y);
           }
-          const float2 ea = ffma2(make_float2(a0, a1), make_float2(sl2, sl2), make_float2(nmu, nmu));
-          const float2 eb = ffma2(make_float2(b0, b1), make_float2(sl2, sl2), make_float2(nmu, nmu));
-          const float2 pa = make_float2(ex2_approx(ea.x), ex2_approx(ea.y));
-          const float2 pb = make_float2(ex2_approx(eb.x), ex2_approx(eb.y));
-          sum2 = fadd2(sum2, fadd2(pa, pb));
-          pk[j] = pack_bf16x2(pa.x, pa.y);
-          pk[16 + j] = pack_bf16x2(pb.x, pb.y);
+        } else {
+          const unsigned long long vm = sl ? vm1 : vm0;
+          const uint32_t lo = (uint32_t)vm, hi = (uint32_t)(vm >> 32);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float a0 = ((lo >> (2 * j)) & 1u) ? __uint_as_float(ra[2 * j]) : -INFINITY;
+            const float a1 = ((lo >> (2 * j + 1)) & 1u) ? __uint_as_float(ra[2 * j + 1]) : -INFINITY;
+            const float b0 = ((hi >> (2 * j)) & 1u) ? __uint_as_float(rb[2 * j]) : -INFINITY;
+            const float b1 = ((hi >> (2 * j + 1)) & 1u) ? __uint_as_float(rb[2 * j + 1]) : -INFINITY;
+            const float2 ea = ffma2(make_float2(a0, a1), make_float2(sl2, sl2), make_float2(nmu, nmu));
+            const float2 eb = ffma2(make_float2(b0, b1), make_float2(sl2, sl2), make_float2(nmu, nmu));
+            const float2 pa = make_float2(ex2_approx(ea.x), ex2_approx(ea.y));
+            const float2 pb = make_float2(ex2_approx(eb.x), ex2_approx(eb.y));
+            sum2 = fadd2(sum2, fadd2(pa, pb));
+            pk[j] = pack_bf16x2(pa.x, pa.y);
+            pk[16 + j] = pack_bf16x2(pb.x, pb.y);
+          }
         }
-        tmem_st32(sS + 32 * h2, pk);
+        tmem_st32(sS + 32 * sl, pk);
       }
       l_run = l_run * alpha + (sum2.x + sum2.y);
       m_run = m_new;
