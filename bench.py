@@ -330,7 +330,7 @@ def run_vs(args, local):
     reps = 2
     ev[0].record(stream)
     for _ in range(reps):
-        dsa.vertical_slash_index(w.q, w.k, p["n_vert"], p["n_slash"], ws=ws)
+        dsa.vertical_slash_index(w.q, w.k, p["n_vert"], p["n_slash"], ws=ws, out=res)
     ev[1].record(stream)
     for _ in range(reps):
         dsa.block_sparse_attn_fwd(w.q, w.k, w.v, res["block_idx"], res["block_cnt"], res["col_idx"],

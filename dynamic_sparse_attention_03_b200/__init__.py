@@ -39,6 +39,7 @@ SYMBOLS = (
     "block_sparse_attn_fwd",
     "sparse_decode_attn",
     "sparse_decode_attn_static",
+    "a_shape_index",
     "dsa_get_status",
     "dsa_block_index_capacity",
     "dsa_version",
@@ -73,6 +74,7 @@ _SIGS = {
     "block_sparse_attn_fwd": [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _I, _P, _P, _I, _P, _P, _SZ, _P],
     "sparse_decode_attn": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P, _SZ, _P],
     "sparse_decode_attn_static": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P],
+    "a_shape_index": [_I, _I, _I, _I, _P, _P, _I, _P],
     "dsa_get_status": [_P, _P],
     "dsa_block_index_capacity": [_I, _I, _I, _F],
     "dsa_version": [],
@@ -221,10 +223,11 @@ def pool_keys(k: torch.Tensor, out: Optional[torch.Tensor] = None, ws: Optional[
 
 def vertical_slash_index(q: torch.Tensor, k: torch.Tensor, n_vert: int, n_slash: int, scale: Optional[float] = None,
                          last_q: int = 64, kcap: Optional[int] = None, ccap: Optional[int] = None,
-                         ws: Optional[Workspace] = None) -> dict:
+                         ws: Optional[Workspace] = None, out: Optional[dict] = None) -> dict:
     """Vertical-slash index and plan.  Returns a dict of int32 tensors:
     vert_idx [Hq][n_vert], slash_off [Hq][n_slash], block_idx [Hq][n/64][kcap],
-    block_cnt, col_idx [Hq][n/64][ccap], col_cnt."""
+    block_cnt, col_idx [Hq][n/64][ccap], col_cnt.  Pass a previous result as
+    `out` to write into the same tensors."""
     _need_cuda(q, k)
     _need_dtype(q, torch.bfloat16, "q")
     _need_dtype(k, torch.bfloat16, "k")
@@ -232,10 +235,14 @@ def vertical_slash_index(q: torch.Tensor, k: torch.Tensor, n_vert: int, n_slash:
     Hkv = k.shape[0]
     nqb = n // 64
     scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dev = q.device
+    if out is not None:
+        kcap = out["block_idx"].shape[-1]
+        ccap = out["col_idx"].shape[-1]
+        _need_cuda(*out.values())
     kcap = min(nqb, 2 * n_slash) if kcap is None else kcap
     ccap = n_vert if ccap is None else ccap
-    dev = q.device
-    out = dict(
+    out = out if out is not None else dict(
         vert_idx=torch.empty((Hq, n_vert), dtype=torch.int32, device=dev),
         slash_off=torch.empty((Hq, n_slash), dtype=torch.int32, device=dev),
         block_idx=torch.empty((Hq, nqb, kcap), dtype=torch.int32, device=dev),
@@ -319,3 +326,16 @@ def sparse_decode_attn_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
         float(scale), _ptr(o), _ptr(sel_idx), _ptr(sel_cnt), kcap, _stream(q.device))
     _check(rc, "sparse_decode_attn_static")
     return (o, sel_idx, sel_cnt) if return_sel else o
+
+
+def a_shape_index(Hq: int, n: int, n_sink: int, n_local: int, device=None):
+    """Static sink + local-window block lists for block_sparse_attn_fwd.
+    Returns (block_idx [Hq][n/64][kcap], block_cnt [Hq][n/64])."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    nqb = n // 64
+    kcap = max(1, min(nqb, n_sink + n_local))
+    bi = torch.empty((Hq, nqb, kcap), dtype=torch.int32, device=dev)
+    bc = torch.empty((Hq, nqb), dtype=torch.int32, device=dev)
+    _check(load_library().a_shape_index(Hq, n, n_sink, n_local, _ptr(bi), _ptr(bc), kcap, _stream(dev)),
+           "a_shape_index")
+    return bi, bc

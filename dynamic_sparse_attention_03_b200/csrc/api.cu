@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/dsa.h"
+#include "ashape.cuh"
 #include "attn_fwd.cuh"
 #include "decode.cuh"
 #include "index_kernels.cuh"
@@ -384,6 +385,19 @@ int block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, 
                             status, st);
   return launch_attn<64>(q, k, v, o, Hq, Hkv, n, scale, block_idx, block_cnt, kcap, col_idx, col_cnt, ccap, lse,
                          status, st);
+}
+
+int a_shape_index(int Hq, int n, int n_sink, int n_local, int32_t* block_idx, int32_t* block_cnt, int kcap,
+                  dsa_stream_t stream) {
+  if (!block_idx || !block_cnt || Hq <= 0 || n <= 0 || n_sink < 0 || n_local < 1) return DSA_ERR_INVALID_ARG;
+  if (n % 64 != 0 || n > kMaxN) return DSA_ERR_UNSUPPORTED;
+  const int nQB = n / 64;
+  const int need = std::min(nQB, n_sink + n_local);
+  if (kcap < need) return DSA_ERR_CAPACITY;
+  const int nrows = Hq * nQB;
+  a_shape_kernel<<<(nrows + 7) / 8, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(nrows, nQB, n_sink, n_local,
+                                                                                     block_idx, block_cnt, kcap);
+  return launch_check();
 }
 
 int sparse_decode_attn(const void* q, const void* k_cache, const void* v_cache, const float* centroids, int B,

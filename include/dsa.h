@@ -134,6 +134,18 @@ int block_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, 
                           size_t* ws_bytes, dsa_stream_t stream);
 
 /*
+ * a_shape_index -- static A-shape block index (MInference 1.0, method
+ * section: the A-shape pattern keeps the first tokens, an attention sink, and
+ * a local window of recent tokens).  Query block qb keeps key blocks
+ * [0, min(n_sink, qb+1)) and [max(0, qb-n_local+1), qb], ascending, -1 padded;
+ * the lists feed block_sparse_attn_fwd unchanged.
+ *  block_idx [Hq][n/64][kcap], block_cnt [Hq][n/64] int32 out;
+ *  kcap >= min(n/64, n_sink + n_local).  n_sink >= 0, n_local >= 1.
+ */
+int a_shape_index(int Hq, int n, int n_sink, int n_local, int32_t* block_idx, int32_t* block_cnt, int kcap,
+                  dsa_stream_t stream);
+
+/*
  * sparse_decode_attn -- one query token per sequence over a fixed KV cache,
  * attending only over the best-ranked 64-token blocks (Squeezed Attention,
  * technical approach, online stage: score the query against every centroid,

@@ -38,3 +38,4 @@ from .vslash import vs_scores, vs_topk, vs_plan, vs_index  # noqa: F401
 from .attention import sparse_attention_rows, sparse_attention, dense_lists  # noqa: F401
 from .decode import decode_centroids, decode_select, decode_attention, sparse_decode  # noqa: F401
 from .ties import compare_index_sets  # noqa: F401
+from .ashape import a_shape_lists  # noqa: F401

@@ -287,3 +287,22 @@ def test_validation_mode_rejects_bad_lists(monkeypatch):
         with pytest.raises(dsa.DSAError) as ei:
             dsa.block_sparse_attn_fwd(q, q, q, b2, c2)
         assert ei.value.rc == -1
+
+
+# ---------------------------------------------------------------- A-shape
+
+@pytest.mark.parametrize("n_sink,n_local", [(1, 4), (2, 7), (0, 3)])
+def test_a_shape_lists_and_attention(n_sink, n_local):
+    Hq, Hkv, n, d = 8, 2, 2048, 128
+    w = synth.make_prefill("llama3-8b-32k-bs10", device=DEV, n=n, Hq=Hq, Hkv=Hkv, d=d, seed=31)
+    bi, bc = dsa.a_shape_index(Hq, n, n_sink, n_local)
+    got = lists_from_gpu(bi, bc)
+    want = oracle.a_shape_lists(n // 64, n_sink, n_local)
+    for h in range(Hq):
+        for qb in range(n // 64):
+            assert got[h][qb].tolist() == want[qb].tolist(), (h, qb)
+    o = dsa.block_sparse_attn_fwd(w.q, w.k, w.v, bi, bc)
+    torch.cuda.synchronize()
+    items = [(h, qb) for h in range(Hq) for qb in range(n // 64)]
+    ref = _ref_attention(w.q, w.k, w.v, got, None, 1 / math.sqrt(d), items)
+    check_attention(o, ref, f"a-shape {n_sink}+{n_local}")

@@ -327,3 +327,17 @@ def test_tie_rule():
     # wrong count, missing forced
     assert oracle.compare_index_sets([0, 1, 2, 8], forced, cand, scores, 3).startswith("MISMATCH")
     assert oracle.compare_index_sets([1, 2, 4, 8], forced, cand, scores, 2).startswith("MISMATCH")
+
+
+# ---------------------------------------------------------------- A-shape
+
+def test_a_shape_closed_form():
+    """Counts written out from the definition: min(qb+1, n_sink + n_local) for
+    every query block (the two ranges overlap once qb < n_sink + n_local)."""
+    lists = oracle.a_shape_lists(40, 2, 5)
+    for qb, sel in lists.items():
+        assert len(sel) == min(qb + 1, 7)
+        assert sel.tolist() == sorted(set(sel.tolist()))
+        assert 0 in sel.tolist() and qb in sel.tolist()
+    assert lists[10].tolist() == [0, 1, 6, 7, 8, 9, 10]
+    assert lists[3].tolist() == [0, 1, 2, 3]
