@@ -207,6 +207,23 @@ def run_ours(args, rank, world, local):
             dsa.block_sparse_attn_fwd(w.q, w.k, w.v, bi, bc, out=o, ws=ws)
         a1.record(stream)
         torch.cuda.synchronize()
+    # cross-layer index reuse (IndexCache's "full" vs "shared" layers): four
+    # layers each estimating their own index, against one estimate shared by
+    # all four; the same tensors stand in for every layer (timing only)
+    r0, r1, r2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    nl = 4
+    r0.record(stream)
+    for _ in range(nl):
+        step()
+    r1.record(stream)
+    dsa.sparse_index_estimate(w.q, w.k, k_fixed=kf, keep_ratio=rho, kcap=kcap, block_idx=bi, block_cnt=bc, ws=ws)
+    for _ in range(nl):
+        dsa.block_sparse_attn_fwd(w.q, w.k, w.v, bi, bc, out=o, ws=ws)
+    r2.record(stream)
+    torch.cuda.synchronize()
+    reuse = {"layers": nl, "index_every_layer_ms": round(r0.elapsed_time(r1), 3),
+             "index_once_ms": round(r1.elapsed_time(r2), 3),
+             "speedup": round(r0.elapsed_time(r1) / r1.elapsed_time(r2), 4)}
     ms = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms, world)
     attn_ms = a0.elapsed_time(a1) / reps
@@ -241,6 +258,7 @@ def run_ours(args, rank, world, local):
                    "parallelism": f"independent layer per GPU x{world}"},
         "breakdown_ms": {"index": round(index_ms, 4), "attention": round(attn_ms, 4)},
         "index_roofline": index_roof,
+        "index_reuse": reuse,
         "effective_flops_per_step": flops,
         "roofline": {"bound": "tensor", "kernel": "bsa_fwd_kernel<128>", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,

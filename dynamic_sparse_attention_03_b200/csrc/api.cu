@@ -288,9 +288,8 @@ int vertical_slash_index(const void* q, const void* k, int Hq, int Hkv, int n, i
   const int ntiles = nQB;
   WsCarve c(ws);
   VSParams p{};
-  p.part = nullptr;
-  uint32_t* status = static_cast<uint32_t*>(c.take(kStatusBytes));
-  (void)status;
+  p.status = static_cast<uint32_t*>(c.take(kStatusBytes));
+  p.zlog = static_cast<float*>(c.take((size_t)Hq * 64 * n * 4));
   p.part = static_cast<float*>(c.take((size_t)Hq * ntiles * 64 * 2 * 4));
   p.lse2 = static_cast<float*>(c.take((size_t)Hq * 64 * 4));
   p.vert = static_cast<float*>(c.take((size_t)Hq * n * 4));
@@ -298,6 +297,9 @@ int vertical_slash_index(const void* q, const void* k, int Hq, int Hkv, int n, i
   p.slash = static_cast<float*>(c.take((size_t)Hq * n * 4));
   p.vsel = vert_idx ? vert_idx : static_cast<int32_t*>(c.take((size_t)Hq * n_vert * 4));
   p.ssel = slash_off ? slash_off : static_cast<int32_t*>(c.take((size_t)Hq * n_slash * 4));
+  p.dbits = static_cast<uint32_t*>(c.take((size_t)Hq * ((nQB + 31) / 32) * 4));
+  p.dlist = static_cast<int32_t*>(c.take((size_t)Hq * nQB * 4));
+  p.dcount = static_cast<int32_t*>(c.take((size_t)Hq * 4));
   if (!ws) {
     *ws_bytes = c.off;
     return DSA_OK;
@@ -321,29 +323,36 @@ int vertical_slash_index(const void* q, const void* k, int Hq, int Hkv, int n, i
   p.ccap = ccap;
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t smem = (2 * (size_t)d * 64 + 64 * 65) * 4;
   int rc;
-  dim3 gt(ntiles, Hq);
-  if (d == 128) {
-    if ((rc = set_smem(vs_pass1_kernel<128>, smem)) || (rc = set_smem(vs_pass2_kernel<128>, smem))) return rc;
-    vs_pass1_kernel<128><<<gt, 256, smem, st>>>(p);
-  } else {
-    if ((rc = set_smem(vs_pass1_kernel<64>, smem)) || (rc = set_smem(vs_pass2_kernel<64>, smem))) return rc;
-    vs_pass1_kernel<64><<<gt, 256, smem, st>>>(p);
+  {
+    CUtensorMap tq, tk;
+    if (!make_tmap(&tq, q, (int64_t)Hq * n, d) || !make_tmap(&tk, k, (int64_t)Hkv * n, d)) return DSA_ERR_CUDA;
+    const dim3 gl((n + 127) / 128, Hkv * ((p.grp + 3) / 4));
+    if (d == 128) {
+      if ((rc = set_smem(vs_logits_kernel<128>, VSLogitLayout<128>::kSmemAlloc))) return rc;
+      vs_logits_kernel<128><<<gl, 256, VSLogitLayout<128>::kSmemAlloc, st>>>(tq, tk, p);
+    } else {
+      if ((rc = set_smem(vs_logits_kernel<64>, VSLogitLayout<64>::kSmemAlloc))) return rc;
+      vs_logits_kernel<64><<<gl, 256, VSLogitLayout<64>::kSmemAlloc, st>>>(tq, tk, p);
+    }
+    if ((rc = launch_check())) return rc;
   }
+  dim3 gt(ntiles, Hq);
+  vs_pass1_kernel<<<gt, 256, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
   vs_lse_kernel<<<Hq, 64, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
-  if (d == 128) vs_pass2_kernel<128><<<gt, 256, smem, st>>>(p);
-  else vs_pass2_kernel<64><<<gt, 256, smem, st>>>(p);
+  vs_pass2_kernel<<<gt, 256, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
   vs_slash_kernel<<<dim3((n + 255) / 256, Hq), 256, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
   vs_topk_kernel<1024><<<dim3(Hq, 2), 1024, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
-  const size_t plan_smem = (size_t)((nQB + 31) / 32) * 4;
-  if ((rc = set_smem(vs_plan_kernel<256>, plan_smem))) return rc;
-  vs_plan_kernel<256><<<dim3(nQB, Hq), 256, plan_smem, st>>>(p);
+  const size_t dist_smem = (size_t)((nQB + 31) / 32) * 4;
+  if ((rc = set_smem(vs_dist_kernel<256>, dist_smem))) return rc;
+  vs_dist_kernel<256><<<Hq, 256, dist_smem, st>>>(p);
+  if ((rc = launch_check())) return rc;
+  vs_plan_kernel<<<(unsigned)(((int64_t)Hq * nQB + 7) / 8), 256, 0, st>>>(p);
   return launch_check();
 }
 

@@ -3,15 +3,18 @@
 // the vertical lines and slash lines; Fig. 4: slash lines as 64x64 blocks,
 // vertical lines as 1x64 column tiles).
 //
-// Rows i_r = n - 64 + r.  Pass 1 computes each row's log-sum-exp over its
-// causal keys; pass 2 recomputes the scores, forms the probabilities
-// P[r][j] = exp(z - lse_r), and sums them per key column (vert) and per
-// diagonal offset o = i_r - j (slash).  Both passes tile the keys in blocks of
-// 64 per CTA (one q-head); every sum runs in a fixed order, so the scores are
-// deterministic run to run.  Then a top-k per head and the per-query-block
-// plan (aligned 64x64 blocks for slashes, column entries for verticals).
+// Rows i_r = n - 64 + r.  The logits z = q_i.k_j * scale (log2 domain) of
+// those rows against every key come from one tcgen05 kernel (a dense
+// product).  Pass 1 then computes each row's log-sum-exp over its causal keys;
+// pass 2 forms the probabilities P[r][j] = 2^(z - lse_r) and sums them per key
+// column (vert) and per diagonal offset o = i_r - j (slash).  Both passes tile
+// the keys in blocks of 64 per CTA (one q-head) and sum in a fixed order, so
+// the scores are deterministic run to run.  Then a top-k per head and the
+// per-query-block plan (aligned 64x64 blocks for slashes, column entries for
+// verticals).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -23,6 +26,8 @@ namespace dsa {
 struct VSParams {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
+  float* zlog;        // [Hq][64][n] logits of the last 64 queries, log2 domain (scale*log2e folded in)
+  uint32_t* status;
   float* part;        // [Hq][ntiles][64][2]  pass-1 (max, sum) per tile and row (log2 domain)
   float* lse2;        // [Hq][64]
   float* vert;        // [Hq][n]
@@ -30,6 +35,9 @@ struct VSParams {
   float* slash;       // [Hq][n]
   int32_t* vsel;      // [Hq][n_vert]
   int32_t* ssel;      // [Hq][n_slash]
+  uint32_t* dbits;    // [Hq][ceil(nQB/32)] block distances reached by kept offsets
+  int32_t* dlist;     // [Hq][nQB] the same distances, ascending
+  int32_t* dcount;    // [Hq]
   int32_t* block_idx;
   int32_t* block_cnt;
   int32_t* col_idx;
@@ -38,71 +46,145 @@ struct VSParams {
   float scale_log2;
 };
 
-// z[r][c] for rows r of the last-64 queries of head h and keys j0+c, c < 64,
-// in the log2 domain (scale * log2 e folded in), -inf where j0 + c > i_r.
-// Shared memory: Qs [D][64], Ks [D][64] fp32 (reduction dim outermost), Z [64][65].
+// ---------------------------------------------------------------- logits on tensor cores
+// Z[h][r][j] = (q_{n-64+r} . k_j) * scale * log2(e) for the last 64 queries
+// of every q-head against all keys of its KV head: a dense product, so it runs
+// on tcgen05.  One CTA per (KV head, group of four q-heads, 128 keys): the
+// four heads' 64 rows form two M=128 tiles (TMA, 128-byte swizzle), the key
+// tile is N=128, fp32 accumulators in TMEM; 8 warps read the accumulators
+// back (one row per thread) and store the scaled row segment.  Causal masking
+// is left to the passes that read Z.
 template <int D>
-__device__ __forceinline__ void vs_logits_tile(const VSParams& p, int h, int tile, float* Qs, float* Ks, float* Z) {
-  const int g = h / p.grp;
+struct VSLogitLayout {
+  static constexpr int NDH = D / 64;
+  static constexpr int kHalf = 16384;        // one d-half of 128 rows x 128 B
+  static constexpr int kTile = NDH * kHalf;
+  static constexpr int kQA = 0, kQB = kTile, kK = 2 * kTile;
+  static constexpr int kBar = 3 * kTile;
+  static constexpr int kBytes = kBar + 64;
+  static constexpr int kSmemAlloc = kBytes + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256, 2)
+    vs_logits_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const VSParams p) {
+  using Lay = VSLogitLayout<D>;
+  extern __shared__ uint8_t vs_smem_raw[];
+  if (status_timed_out(p.status)) return;
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(vs_smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t bar_full = sb + Lay::kBar, bar_mma = bar_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kBar + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kBar + 20);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nquads = (p.grp + 3) / 4;
+  const int g = blockIdx.y / nquads, quad = blockIdx.y % nquads;
+  const int h0 = g * p.grp + 4 * quad;
+  const int nh = min(4, p.grp - 4 * quad);
+  const int j0 = blockIdx.x * 128;
+  if (threadIdx.x == 0) {
+    mbar_init(bar_full, 1);
+    mbar_init(bar_mma, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const AbortState ab{abort_flag, p.status};
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar_full, (uint32_t)(3 * Lay::kTile));
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh) {
+      const int h = h0 + min(hh, nh - 1);
+#pragma unroll
+      for (int dh = 0; dh < Lay::NDH; ++dh)
+        tma_load_2d(sb + (hh >> 1) * Lay::kTile + dh * Lay::kHalf + (hh & 1) * 8192, &tmQ, dh * 64,
+                    h * p.n + p.n - 64, bar_full);
+    }
+#pragma unroll
+    for (int dh = 0; dh < Lay::NDH; ++dh) {
+      tma_load_2d(sb + Lay::kK + dh * Lay::kHalf, &tmK, dh * 64, g * p.n + j0, bar_full);
+      tma_load_2d(sb + Lay::kK + dh * Lay::kHalf + 8192, &tmK, dh * 64, g * p.n + j0 + 64, bar_full);
+    }
+    if (mbar_wait(bar_full, 0, ab)) {
+      tc_fence_after();
+      const uint32_t idesc = umma_idesc_bf16(128, 128, 0);
+#pragma unroll
+      for (int tile = 0; tile < 2; ++tile) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = umma_desc_sw128(sb + tile * Lay::kTile + (kk >> 2) * Lay::kHalf + (kk & 3) * 32, 16, 1024);
+          const uint64_t b = umma_desc_sw128(sb + Lay::kK + (kk >> 2) * Lay::kHalf + (kk & 3) * 32, 16, 1024);
+          umma_bf16_ss(tmem + 128u * (uint32_t)tile, a, b, idesc, kk > 0 ? 1u : 0u);
+        }
+      }
+    }
+    umma_commit(bar_mma);
+  }
+  // epilogue: warp w reads TMEM lane quarter w%4 of tile w/4
+  const int tile = warp >> 2, q4 = warp & 3;
+  const int row = q4 * 32 + lane;
+  const int hh = 2 * tile + (row >> 6), r = row & 63;
+  const bool ok = mbar_wait_warp(bar_mma, 0, ab);
+  if (ok && hh < nh) {
+    tc_fence_after();
+    float* dst = p.zlog + ((size_t)(h0 + hh) * 64 + r) * p.n + j0;
+    const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16) + 128u * (uint32_t)tile;
+    const int nchunk = min(128, p.n - j0) / 32;   // the last tile of an n % 128 == 64 sequence has 64 keys
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c >= nchunk) break;
+      uint32_t v[32];
+      tmem_ld32(ta + 32 * c, v);
+      tmem_wait_ld();
+      reg_fence(v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 w = make_float4(__uint_as_float(v[4 * q]) * p.scale_log2, __uint_as_float(v[4 * q + 1]) * p.scale_log2,
+                                     __uint_as_float(v[4 * q + 2]) * p.scale_log2,
+                                     __uint_as_float(v[4 * q + 3]) * p.scale_log2);
+        *reinterpret_cast<float4*>(dst + 32 * c + 4 * q) = w;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// z[r][c] (log2 domain) of rows r of the last-64 queries of head h and keys
+// j0+c, c < 64, read from the logits above; -inf where j0 + c > i_r.
+__device__ __forceinline__ void vs_load_tile(const VSParams& p, int h, int tile, float* Z) {
   const int j0 = tile * 64;
   const int i0 = p.n - 64;
-  const __nv_bfloat16* qsrc = p.q + ((size_t)h * p.n + i0) * D;
-  const __nv_bfloat16* ksrc = p.k + ((size_t)g * p.n + j0) * D;
-  for (int idx = threadIdx.x; idx < 64 * D / 8; idx += 256) {
-    const int m = idx / (D / 8), k8 = (idx % (D / 8)) * 8;
-    const uint4 qa = __ldg(reinterpret_cast<const uint4*>(qsrc + (size_t)m * D + k8));
-    const uint4 ka = __ldg(reinterpret_cast<const uint4*>(ksrc + (size_t)m * D + k8));
-    const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qa);
-    const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&ka);
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const float2 qf = __bfloat1622float2(q2[a]);
-      const float2 kf = __bfloat1622float2(k2[a]);
-      Qs[(k8 + 2 * a) * 64 + m] = qf.x;
-      Qs[(k8 + 2 * a + 1) * 64 + m] = qf.y;
-      Ks[(k8 + 2 * a) * 64 + m] = kf.x;
-      Ks[(k8 + 2 * a + 1) * 64 + m] = kf.y;
-    }
-  }
-  __syncthreads();
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-#pragma unroll 8
-  for (int kk = 0; kk < D; ++kk) {
-    const float4 av = *reinterpret_cast<const float4*>(Qs + kk * 64 + ty * 4);
-    const float4 bv = *reinterpret_cast<const float4*>(Ks + kk * 64 + tx * 4);
-    const float ar[4] = {av.x, av.y, av.z, av.w};
-    const float br[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(ar[a], br[b], acc[a][b]);
-  }
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int r = ty * 4 + a;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int c = tx * 4 + b;
-      Z[r * 65 + c] = (j0 + c <= i0 + r) ? acc[a][b] * p.scale_log2 : -INFINITY;
-    }
+  const float* src = p.zlog + (size_t)h * 64 * p.n + j0;
+  for (int x = threadIdx.x; x < 64 * 16; x += 256) {
+    const int r = x >> 4, c4 = (x & 15) * 4;
+    const float4 v = __ldg(reinterpret_cast<const float4*>(src + (size_t)r * p.n + c4));
+    Z[r * 65 + c4 + 0] = (j0 + c4 + 0 <= i0 + r) ? v.x : -INFINITY;
+    Z[r * 65 + c4 + 1] = (j0 + c4 + 1 <= i0 + r) ? v.y : -INFINITY;
+    Z[r * 65 + c4 + 2] = (j0 + c4 + 2 <= i0 + r) ? v.z : -INFINITY;
+    Z[r * 65 + c4 + 3] = (j0 + c4 + 3 <= i0 + r) ? v.w : -INFINITY;
   }
   __syncthreads();
 }
 
 // Pass 1: per (tile, head): row max and sum of exp2 over the tile's keys.
-template <int D>
 __global__ void __launch_bounds__(256) vs_pass1_kernel(const VSParams p) {
-  extern __shared__ __align__(16) float vsm[];
-  float* Qs = vsm;
-  float* Ks = Qs + D * 64;
-  float* Z = Ks + D * 64;
+  __shared__ __align__(16) float Z[64 * 65];
   const int tile = blockIdx.x, h = blockIdx.y;
-  vs_logits_tile<D>(p, h, tile, Qs, Ks, Z);
+  vs_load_tile(p, h, tile, Z);
   // 4 threads per row
   const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
   float mx = -INFINITY;
@@ -137,14 +219,10 @@ __global__ void __launch_bounds__(64) vs_lse_kernel(const VSParams p) {
 
 // Pass 2: probabilities of the tile; column sums (complete) and diagonal
 // partial sums of the tile's 127 offsets.
-template <int D>
 __global__ void __launch_bounds__(256) vs_pass2_kernel(const VSParams p) {
-  extern __shared__ __align__(16) float vsm[];
-  float* Qs = vsm;
-  float* Ks = Qs + D * 64;
-  float* Z = Ks + D * 64;
+  __shared__ __align__(16) float Z[64 * 65];
   const int tile = blockIdx.x, h = blockIdx.y;
-  vs_logits_tile<D>(p, h, tile, Qs, Ks, Z);
+  vs_load_tile(p, h, tile, Z);
   for (int x = threadIdx.x; x < 64 * 64; x += 256) {
     const int r = x >> 6, c = x & 63;
     const float z = Z[r * 65 + c];
@@ -197,69 +275,97 @@ __global__ void __launch_bounds__(NT) vs_topk_kernel(const VSParams p) {
   }
 }
 
-// Plan for (qb, h): blocks touched by the kept offsets, and kept columns whose
-// block is not among them.
+// Block distances of a head's kept offsets: a kept offset o reaches key
+// blocks qb - floor(o/64) and qb - ceil(o/64) of query block qb exactly when
+// that distance is <= qb (then o <= 64*qb + 63 holds).  So every query
+// block's block list is {qb - delta : delta in D, delta <= qb} for one
+// per-head distance set D.  One CTA per head builds D as a bitmap and as an
+// ascending list.
 template <int NT>
-__global__ void __launch_bounds__(NT) vs_plan_kernel(const VSParams p) {
-  extern __shared__ __align__(16) uint32_t bits[];   // nQB bits
+__global__ void __launch_bounds__(NT) vs_dist_kernel(const VSParams p) {
+  extern __shared__ __align__(16) uint32_t dbits_s[];   // nQB bits
   __shared__ SelectSmem sm;
-  const int qb = blockIdx.x, h = blockIdx.y;
+  const int h = blockIdx.x;
   const int nwords = (p.nQB + 31) >> 5;
-  for (int w = threadIdx.x; w < nwords; w += NT) bits[w] = 0u;
+  for (int w = threadIdx.x; w < nwords; w += NT) dbits_s[w] = 0u;
   __syncthreads();
-  const int last = 64 * qb + 63;
   const int32_t* so = p.ssel + (size_t)h * p.n_slash;
   for (int x = threadIdx.x; x < p.n_slash; x += NT) {
     const int o = so[x];
-    if (o < 0 || o > last) continue;
-    const int near = qb - (o >> 6);
-    const int far = qb - ((o + 63) >> 6);
-    atomicOr(&bits[near >> 5], 1u << (near & 31));
-    if (far >= 0) atomicOr(&bits[far >> 5], 1u << (far & 31));
+    if (o < 0) continue;
+    const int near = o >> 6, far = (o + 63) >> 6;
+    if (near < p.nQB) atomicOr(&dbits_s[near >> 5], 1u << (near & 31));
+    if (far < p.nQB) atomicOr(&dbits_s[far >> 5], 1u << (far & 31));
   }
   __syncthreads();
-  // blocks: ordered compaction over positions 0..qb
-  {
-    const int P = qb + 1;
-    const int per = (P + NT - 1) / NT;
-    const int p0 = min(P, (int)threadIdx.x * per), p1 = min(P, p0 + per);
-    int kept = 0;
-    for (int x = p0; x < p1; ++x) kept += (bits[x >> 5] >> (x & 31)) & 1u;
-    int total;
-    int off = block_excl_scan<NT>(kept, sm, total);
-    int32_t* out = p.block_idx + ((size_t)h * p.nQB + qb) * p.kcap;
-    for (int x = p0; x < p1; ++x)
-      if ((bits[x >> 5] >> (x & 31)) & 1u) {
-        if (off < p.kcap) out[off] = x;
-        ++off;
-      }
-    for (int x = total + (int)threadIdx.x; x < p.kcap; x += NT) out[x] = -1;
-    if (threadIdx.x == 0) p.block_cnt[(size_t)h * p.nQB + qb] = min(total, p.kcap);
+  uint32_t* dbits = p.dbits + (size_t)h * nwords;
+  for (int w = threadIdx.x; w < nwords; w += NT) dbits[w] = dbits_s[w];
+  const int per = (p.nQB + NT - 1) / NT;
+  const int p0 = min(p.nQB, (int)threadIdx.x * per), p1 = min(p.nQB, p0 + per);
+  int kept = 0;
+  for (int x = p0; x < p1; ++x) kept += (dbits_s[x >> 5] >> (x & 31)) & 1u;
+  int total;
+  int off = block_excl_scan<NT>(kept, sm, total);
+  int32_t* dlist = p.dlist + (size_t)h * p.nQB;
+  for (int x = p0; x < p1; ++x)
+    if ((dbits_s[x >> 5] >> (x & 31)) & 1u) dlist[off++] = x;
+  if (threadIdx.x == 0) p.dcount[h] = total;
+}
+
+// Plan for (h, qb), one warp each: blocks qb - delta for the distances
+// delta <= qb in ascending block order, then the kept columns j <= 64*qb+63
+// whose block's distance qb - j/64 is not in D, in list order.
+__global__ void __launch_bounds__(256) vs_plan_kernel(const VSParams p) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= p.Hq * p.nQB) return;
+  const int h = row / p.nQB, qb = row % p.nQB;
+  const int32_t* dlist = p.dlist + (size_t)h * p.nQB;
+  const int dc = p.dcount[h];
+  const uint32_t* dbits = p.dbits + (size_t)h * ((p.nQB + 31) >> 5);
+  // number of distances <= qb (dlist ascending): binary search by every lane
+  int lo = 0, hi = dc;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (dlist[mid] <= qb) lo = mid + 1;
+    else hi = mid;
   }
-  // columns: kept j <= last with block not selected, in list order
-  {
-    const int32_t* vi = p.vsel + (size_t)h * p.n_vert;
-    const int P = p.n_vert;
-    const int per = (P + NT - 1) / NT;
-    const int p0 = min(P, (int)threadIdx.x * per), p1 = min(P, p0 + per);
-    int kept = 0;
-    for (int x = p0; x < p1; ++x) {
-      const int j = vi[x];
-      kept += (j >= 0 && j <= last && !((bits[j >> 11] >> ((j >> 6) & 31)) & 1u));
-    }
-    int total;
-    int off = block_excl_scan<NT>(kept, sm, total);
-    int32_t* out = p.col_idx + ((size_t)h * p.nQB + qb) * p.ccap;
-    for (int x = p0; x < p1; ++x) {
-      const int j = vi[x];
-      if (j >= 0 && j <= last && !((bits[j >> 11] >> ((j >> 6) & 31)) & 1u)) {
-        if (off < p.ccap) out[off] = j;
-        ++off;
-      }
-    }
-    for (int x = total + (int)threadIdx.x; x < p.ccap; x += NT) out[x] = -1;
-    if (threadIdx.x == 0) p.col_cnt[(size_t)h * p.nQB + qb] = min(total, p.ccap);
+  const int c = min(lo, p.kcap);
+  int32_t* bout = p.block_idx + (size_t)row * p.kcap;
+  for (int k = lane; k < p.kcap; k += 32) bout[k] = k < c ? qb - dlist[lo - 1 - k] : -1;
+  if (lane == 0) p.block_cnt[row] = c;
+  // columns: the kept columns are ascending, so j <= 64*qb+63 is a prefix
+  const int32_t* vi = p.vsel + (size_t)h * p.n_vert;
+  const int last = 64 * qb + 63;
+  lo = 0;
+  hi = p.n_vert;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (vi[mid] <= last) lo = mid + 1;
+    else hi = mid;
   }
+  const int m = lo;
+  int32_t* cout = p.col_idx + (size_t)row * p.ccap;
+  const unsigned lt = (1u << lane) - 1u;
+  int off = 0;
+  for (int base = 0; base < m; base += 32) {
+    const int x = base + lane;
+    bool keep = false;
+    int j = 0;
+    if (x < m) {
+      j = vi[x];
+      const int dist = qb - (j >> 6);
+      keep = !((dbits[dist >> 5] >> (dist & 31)) & 1u);
+    }
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
+    if (keep) {
+      const int slot = off + __popc(bal & lt);
+      if (slot < p.ccap) cout[slot] = j;
+    }
+    off += __popc(bal);
+  }
+  for (int k = off + lane; k < p.ccap; k += 32) cout[k] = -1;
+  if (lane == 0) p.col_cnt[row] = min(off, p.ccap);
 }
 
 }  // namespace dsa

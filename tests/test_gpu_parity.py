@@ -166,8 +166,9 @@ def test_attention_invariants():
 
 # ---------------------------------------------------------------- vertical-slash
 
-def test_vs_index_plan_and_attention_small():
-    Hq, Hkv, n, d = 4, 2, 2048, 128
+@pytest.mark.parametrize("n", [2048, 1984])
+def test_vs_index_plan_and_attention_small(n):
+    Hq, Hkv, d = 4, 2, 128
     w = synth.make_prefill("llama3-8b-128k-vs", device=DEV, n=n, Hq=Hq, Hkv=Hkv, d=d, seed=21)
     n_vert, n_slash = 200, 300
     res = dsa.vertical_slash_index(w.q, w.k, n_vert, n_slash)
