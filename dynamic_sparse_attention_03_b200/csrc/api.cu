@@ -79,6 +79,20 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t rows, int d) {
   return r == CUDA_SUCCESS;
 }
 
+// 2D fp32 view [rows][d] with a 32-float (128-byte) x box_rows box and 128-byte swizzle.
+bool make_tmap_f32(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 4};
+  cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool validate_env() {
   const char* v = std::getenv("DSA_VALIDATE");
   return v && v[0] == '1';
@@ -221,31 +235,40 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   }
   WsCarve c(ws);
   uint32_t* status = static_cast<uint32_t*>(c.take(kStatusBytes));
-  float* qbar = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hq * nQB * d * 4));
-  float* kbar = pooled_k ? pooled_k : static_cast<float*>(c.take((size_t)Hkv * nQB * d * 4));
+  // TF32 hi/lo halves of the pooled means, the operands of the tensor-core scores
+  float* q_hi = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hq * nQB * d * 4));
+  float* q_lo = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hq * nQB * d * 4));
+  float* k_hi = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hkv * nQB * d * 4));
+  float* k_lo = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hkv * nQB * d * 4));
+  float* kbar = pooled_k;
   float* scores = pool_only ? nullptr : static_cast<float*>(c.take((size_t)chunk * nQB * nQB * 4));
   if (!ws) {
     *ws_bytes = c.off;
     return DSA_OK;
   }
   if (*ws_bytes < c.off) return DSA_ERR_INVALID_ARG;
-  (void)status;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
-  if (d == 128) pool_blocks_kernel<128><<<(unsigned)((int64_t)Hkv * nQB), 256, 0, st>>>(kb, kbar, (int64_t)Hkv * nQB);
-  else pool_blocks_kernel<64><<<(unsigned)((int64_t)Hkv * nQB), 256, 0, st>>>(kb, kbar, (int64_t)Hkv * nQB);
+  const int64_t nkb = (int64_t)Hkv * nQB, nqb = (int64_t)Hq * nQB;
+  if (d == 128) pool_blocks_kernel<128><<<(unsigned)nkb, 256, 0, st>>>(kb, kbar, nkb, k_hi, k_lo);
+  else pool_blocks_kernel<64><<<(unsigned)nkb, 256, 0, st>>>(kb, kbar, nkb, k_hi, k_lo);
   if (int rc = launch_check()) return rc;
   if (pool_only) return DSA_OK;
   const auto* qp = static_cast<const __nv_bfloat16*>(q);
-  if (d == 128) pool_blocks_kernel<128><<<(unsigned)((int64_t)Hq * nQB), 256, 0, st>>>(qp, qbar, (int64_t)Hq * nQB);
-  else pool_blocks_kernel<64><<<(unsigned)((int64_t)Hq * nQB), 256, 0, st>>>(qp, qbar, (int64_t)Hq * nQB);
+  if (d == 128) pool_blocks_kernel<128><<<(unsigned)nqb, 256, 0, st>>>(qp, nullptr, nqb, q_hi, q_lo);
+  else pool_blocks_kernel<64><<<(unsigned)nqb, 256, 0, st>>>(qp, nullptr, nqb, q_hi, q_lo);
   if (int rc = launch_check()) return rc;
-  const int ntr = (nQB + kScoreTile - 1) / kScoreTile;
-  const unsigned ntiles = (unsigned)(ntr * (ntr + 1) / 2);
+  CUtensorMap tqh, tql, tkh, tkl;
+  if (!make_tmap_f32(&tqh, q_hi, nqb, d, 128) || !make_tmap_f32(&tql, q_lo, nqb, d, 128) ||
+      !make_tmap_f32(&tkh, k_hi, nkb, d, 64) || !make_tmap_f32(&tkl, k_lo, nkb, d, 64))
+    return DSA_ERR_CUDA;
+  const int nrt = (nQB + 127) / 128;   // row tiles of 128 query blocks; row tile r has 2r+2 column tiles of 64
+  const unsigned ntiles = (unsigned)(nrt * (nrt + 1));
   constexpr int kSelWarps = 4;
   const bool warp_select = nQB <= 4096;   // a row per warp in shared memory
   const size_t sel_smem = warp_select ? (size_t)kSelWarps * nQB * 4 : (size_t)nQB * 4;
-  int rc = (d == 128) ? set_smem(block_scores_kernel<128>, kScoreSmem) : set_smem(block_scores_kernel<64>, kScoreSmem);
+  int rc = (d == 128) ? set_smem(block_scores_tc_kernel<128>, ScoreTcLayout<128>::kSmemAlloc)
+                      : set_smem(block_scores_tc_kernel<64>, ScoreTcLayout<64>::kSmemAlloc);
   if (rc) return rc;
   if (warp_select) {
     if ((rc = set_smem(block_select_warp_kernel<kSelWarps>, sel_smem))) return rc;
@@ -257,8 +280,12 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   for (int h0 = 0; h0 < Hq; h0 += chunk) {
     const int hc = std::min(chunk, Hq - h0);
     dim3 gs(ntiles, hc);
-    if (d == 128) block_scores_kernel<128><<<gs, 256, kScoreSmem, st>>>(qbar, kbar, scores, nQB, h0, grp);
-    else block_scores_kernel<64><<<gs, 256, kScoreSmem, st>>>(qbar, kbar, scores, nQB, h0, grp);
+    if (d == 128)
+      block_scores_tc_kernel<128><<<gs, 128, ScoreTcLayout<128>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, scores, nQB, h0,
+                                                                                   grp, status);
+    else
+      block_scores_tc_kernel<64><<<gs, 128, ScoreTcLayout<64>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, scores, nQB, h0,
+                                                                                 grp, status);
     if ((rc = launch_check())) return rc;
     if (warp_select) {
       const int nrows = hc * nQB;

@@ -20,9 +20,20 @@ constexpr int kBlock = 64;
 // fp32 mean of the 64 rows.  Each thread loads 16-byte vectors; the 64 rows
 // are summed as (rows r, r+RP, ...) per thread then over the RP row groups in
 // a fixed order, so the result is deterministic.
+// Optionally (out_hi/out_lo not null) also writes the mean split for the
+// tensor-core scores: hi = the mean rounded to TF32, lo = mean - hi (exact in
+// fp32), so hi + lo carries the full fp32 mean.
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) pool_blocks_kernel(const __nv_bfloat16* __restrict__ x,
-                                                           float* __restrict__ out, int64_t nblocks) {
+                                                           float* __restrict__ out, int64_t nblocks,
+                                                           float* __restrict__ out_hi = nullptr,
+                                                           float* __restrict__ out_lo = nullptr) {
   constexpr int VPR = D / 8;          // 16-byte vectors per row
   constexpr int RP = 256 / VPR;       // rows per pass
   constexpr int PASSES = kBlock / RP;
@@ -54,115 +65,160 @@ __global__ void __launch_bounds__(256) pool_blocks_kernel(const __nv_bfloat16* _
     float s = 0.f;
 #pragma unroll
     for (int r = 0; r < RP; ++r) s += part[r][c];
-    out[blk * D + c] = s * (1.0f / kBlock);
+    const float mean = s * (1.0f / kBlock);
+    if (out) out[blk * D + c] = mean;
+    if (out_hi) {
+      const float hi = tf32_round(mean);
+      out_hi[blk * D + c] = hi;
+      out_lo[blk * D + c] = mean - hi;
+    }
   }
 }
 
-// ---------------------------------------------------------------- pooled scores
-// S[hl][i][j] = Q̄[h0+hl][i] · K̄[g][j] for the lower-triangular 128x128 tiles
-// (tile column <= tile row) of every head of the chunk; fp32 FMA.  256
-// threads, each computing an 8x8 sub-tile (rows ty*4+{0..3} and 64+ty*4+{0..3},
-// columns likewise with tx), so four 16-byte shared loads feed 64 FMAs.  The
-// reduction dimension is staged in chunks of 32, double-buffered through
-// registers, transposed so it is outermost in shared memory.
-constexpr int kScoreTile = 128;
-constexpr int kScoreKC = 32;
-constexpr int kScoreLd = 132;   // padded row of the transposed stage
-constexpr size_t kScoreSmem = 2 * 2 * kScoreKC * kScoreLd * sizeof(float);
+// ---------------------------------------------------------------- pooled scores on tensor cores
+// S = Q̄ K̄^T with fp32-level accuracy from three TF32 products,
+// S ~= Qhi Khi + Qhi Klo + Qlo Khi (the dropped Qlo Klo term is ~2^-22
+// relative), accumulated in fp32 in TMEM.  One CTA (4 warps) per
+// (head, 128 query blocks, 64 key blocks) tile on or below the diagonal: the
+// reduction dimension d streams in chunks of 32 floats (one 128-byte swizzle
+// atom) through a 2-stage TMA ring; thread 0 issues the MMAs; the 4 warps read
+// the accumulators back, one query block per thread, and store the row.
+template <int D>
+struct ScoreTcLayout {
+  static constexpr int kA = 128 * 128;            // 128 rows x 32 fp32
+  static constexpr int kB = 64 * 128;             // 64 rows x 32 fp32
+  static constexpr int kStage = 2 * kA + 2 * kB;  // hi and lo of both operands
+  static constexpr int kBar = 2 * kStage;
+  static constexpr int kBytes = kBar + 64;
+  static constexpr int kSmemAlloc = kBytes + 1024;
+  static constexpr int NCH = D / 32;
+};
+
+__host__ __device__ constexpr uint32_t umma_idesc_tf32(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_tf32_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 template <int D>
-__global__ void __launch_bounds__(256) block_scores_kernel(const float* __restrict__ qbar,
-                                                            const float* __restrict__ kbar,
-                                                            float* __restrict__ S, int nQB, int h0,
-                                                            int grp) {
-  extern __shared__ __align__(16) float sm_scores[];
-  // [buf][A/B][k][m]
-  auto stage = [&](int buf, int ab) { return sm_scores + ((buf * 2 + ab) * kScoreKC) * kScoreLd; };
+__global__ void __launch_bounds__(128, 2)
+    block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmQl,
+                           const __grid_constant__ CUtensorMap tmKh, const __grid_constant__ CUtensorMap tmKl,
+                           float* __restrict__ S, int nQB, int h0, int grp, uint32_t* status) {
+  using Lay = ScoreTcLayout<D>;
+  extern __shared__ uint8_t sc_smem_raw[];
+  if (status_timed_out(status)) return;
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sc_smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t bar0 = sb + Lay::kBar;   // full[2], empty[2], done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kBar + 40);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kBar + 44);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hl = blockIdx.y, h = h0 + hl, g = h / grp;
-  // triangular tile index -> (rt, ct), ct <= rt
+  // tile x -> (rt, ct): row tile rt (128 query blocks) has column tiles ct = 0 .. 2*rt+1 (64 each)
   const int x = blockIdx.x;
-  int rt = (int)((sqrtf(8.f * (float)x + 1.f) - 1.f) * 0.5f);
-  while ((rt + 1) * (rt + 2) / 2 <= x) ++rt;
-  while (rt * (rt + 1) / 2 > x) --rt;
-  const int ct = x - rt * (rt + 1) / 2;
-  const int tid = threadIdx.x;
-  const float* qa = qbar + ((size_t)h * nQB + (size_t)rt * kScoreTile) * D;
-  const float* kb = kbar + ((size_t)g * nQB + (size_t)ct * kScoreTile) * D;
-  // loads of one chunk: 128 rows x 32 floats per operand, 4 float4 per thread each
-  float4 ra[4], rb[4];
-  auto load = [&](int c) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int idx = tid + 256 * q;
-      const int m = idx >> 3, k4 = (idx & 7) * 4;
-      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      ra[q] = (rt * kScoreTile + m < nQB) ? *reinterpret_cast<const float4*>(qa + (size_t)m * D + c * kScoreKC + k4) : z;
-      rb[q] = (ct * kScoreTile + m < nQB) ? *reinterpret_cast<const float4*>(kb + (size_t)m * D + c * kScoreKC + k4) : z;
-    }
-  };
-  auto store = [&](int buf) {
-    float* As = stage(buf, 0);
-    float* Bs = stage(buf, 1);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int idx = tid + 256 * q;
-      const int m = idx >> 3, k4 = (idx & 7) * 4;
-      As[(k4 + 0) * kScoreLd + m] = ra[q].x; As[(k4 + 1) * kScoreLd + m] = ra[q].y;
-      As[(k4 + 2) * kScoreLd + m] = ra[q].z; As[(k4 + 3) * kScoreLd + m] = ra[q].w;
-      Bs[(k4 + 0) * kScoreLd + m] = rb[q].x; Bs[(k4 + 1) * kScoreLd + m] = rb[q].y;
-      Bs[(k4 + 2) * kScoreLd + m] = rb[q].z; Bs[(k4 + 3) * kScoreLd + m] = rb[q].w;
-    }
-  };
-  const int tx = tid & 15, ty = tid >> 4;
-  float acc[8][8];
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-  constexpr int NCH = D / kScoreKC;
-  load(0);
-  store(0);
-  __syncthreads();
-#pragma unroll 1
-  for (int c = 0; c < NCH; ++c) {
-    if (c + 1 < NCH) load(c + 1);
-    const float* As = stage(c & 1, 0);
-    const float* Bs = stage(c & 1, 1);
-#pragma unroll 4
-    for (int k = 0; k < kScoreKC; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4*>(As + k * kScoreLd + ty * 4);
-      const float4 a1 = *reinterpret_cast<const float4*>(As + k * kScoreLd + 64 + ty * 4);
-      const float4 b0 = *reinterpret_cast<const float4*>(Bs + k * kScoreLd + tx * 4);
-      const float4 b1 = *reinterpret_cast<const float4*>(Bs + k * kScoreLd + 64 + tx * 4);
-      const float ar[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float br[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(ar[a], br[b], acc[a][b]);
-    }
-    if (c + 1 < NCH) store((c + 1) & 1);
-    __syncthreads();
+  int rt = (int)((sqrtf(4.f * (float)x + 1.f) - 1.f) * 0.5f);
+  while ((rt + 1) * (rt + 2) <= x) ++rt;
+  while (rt * (rt + 1) > x) --rt;
+  const int ct = x - rt * (rt + 1);
+  if (ct * 64 >= nQB) return;   // whole tile past the last key block (ragged last row tile)
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 5; ++b) mbar_init(bar0 + 8u * b, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  float* out = S + (size_t)hl * nQB * nQB;
-  const bool vec = (nQB & 3) == 0;
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const AbortState ab{abort_flag, status};
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 16u + 8u * s; };
+  const uint32_t done = bar0 + 32u;
+  const int arow = h * nQB + rt * 128, brow = g * nQB + ct * 64;
+  if (threadIdx.x == 0) {
+    auto load = [&](int c) {
+      const uint32_t st = sb + (c & 1) * Lay::kStage;
+      mbar_arrive_expect_tx(full(c & 1), (uint32_t)Lay::kStage);
+      tma_load_2d(st, &tmQh, c * 32, arow, full(c & 1));
+      tma_load_2d(st + Lay::kA, &tmQl, c * 32, arow, full(c & 1));
+      tma_load_2d(st + 2 * Lay::kA, &tmKh, c * 32, brow, full(c & 1));
+      tma_load_2d(st + 2 * Lay::kA + Lay::kB, &tmKl, c * 32, brow, full(c & 1));
+    };
+    load(0);
+    if (Lay::NCH > 1) load(1);
+    const uint32_t idesc = umma_idesc_tf32(128, 64);
+    bool ok = true;
+    for (int c = 0; c < Lay::NCH && ok; ++c) {
+      if (!mbar_wait(full(c & 1), (c >> 1) & 1, ab)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t st = sb + (c & 1) * Lay::kStage;
+      const uint32_t aH = st, aL = st + Lay::kA, bH = st + 2 * Lay::kA, bL = bH + Lay::kB;
 #pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int i = rt * kScoreTile + (a < 4 ? ty * 4 + a : 64 + ty * 4 + a - 4);
-    if (i >= nQB) continue;
-#pragma unroll
-    for (int hb = 0; hb < 2; ++hb) {
-      const int j0 = ct * kScoreTile + hb * 64 + tx * 4;
-      float* dst = out + (size_t)i * nQB + j0;
-      if (vec && j0 + 3 < nQB) {
-        *reinterpret_cast<float4*>(dst) =
-            make_float4(acc[a][hb * 4], acc[a][hb * 4 + 1], acc[a][hb * 4 + 2], acc[a][hb * 4 + 3]);
-      } else {
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          if (j0 + b < nQB) dst[b] = acc[a][hb * 4 + b];
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t ko = kk * 32;   // 8 fp32 per step
+        const uint32_t acc0 = (c > 0 || kk > 0) ? 1u : 0u;
+        umma_tf32_ss(tmem, umma_desc_sw128(aH + ko, 16, 1024), umma_desc_sw128(bH + ko, 16, 1024), idesc, acc0);
+        umma_tf32_ss(tmem, umma_desc_sw128(aH + ko, 16, 1024), umma_desc_sw128(bL + ko, 16, 1024), idesc, 1u);
+        umma_tf32_ss(tmem, umma_desc_sw128(aL + ko, 16, 1024), umma_desc_sw128(bH + ko, 16, 1024), idesc, 1u);
+      }
+      umma_commit(empty(c & 1));
+      if (c + 2 < Lay::NCH) {
+        if (!mbar_wait(empty(c & 1), (c >> 1) & 1, ab)) { ok = false; break; }
+        load(c + 2);
       }
     }
+    umma_commit(done);
+  }
+  const bool ok = mbar_wait_warp(done, 0, ab);
+  if (ok) {
+    tc_fence_after();
+    const int i = rt * 128 + warp * 32 + lane;
+    const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16);
+    float* out = S + ((size_t)hl * nQB + i) * nQB + ct * 64;
+    const bool vec = (nQB & 3) == 0;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      uint32_t v[32];
+      tmem_ld32(ta + 32 * cc, v);
+      tmem_wait_ld();
+      reg_fence(v);
+      if (i < nQB) {
+        const int j0 = ct * 64 + 32 * cc;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int j = j0 + 4 * q;
+          if (vec && j + 3 < nQB) {
+            *reinterpret_cast<float4*>(out + 32 * cc + 4 * q) =
+                make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
+                            __uint_as_float(v[4 * q + 3]));
+          } else {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              if (j + b < nQB) out[32 * cc + 4 * q + b] = __uint_as_float(v[4 * q + b]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
   }
 }
 

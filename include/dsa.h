@@ -80,8 +80,10 @@ enum {
  *             DSA_ERR_CAPACITY).
  *  pooled_k   optional [Hkv][n/64][d] fp32 out: the per-block mean keys.
  *             Required in pool-only mode.
- *  Ranking uses fp32 scores; the remaining candidates of query block i are
- *  blocks 1..i-1.
+ *  Ranking uses fp32-accurate scores (three TF32 tensor-core products of the
+ *  split means, |error| ~ 2^-21 of |Q̄||K̄|); the remaining candidates of query
+ *  block i are blocks 1..i-1.  A bounded wait that expires sets the workspace
+ *  status word (DSA_ERR_TIMEOUT through dsa_get_status).
  */
 int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, int d, int block,
                           int k_fixed, float keep_ratio, int32_t* block_idx, int32_t* block_cnt,
