@@ -269,6 +269,33 @@ def run_ours(args, rank, world, local):
     return res, (w, bi, bc, kf, rho, kcap, flops, ws)
 
 
+def run_dense(args, ctx, local, attn_flops_ms):
+    """Dense causal attention through torch SDPA on the same tensors, for context
+    (the pages' "speedup over dense FlashAttention" framing).  Library code, not
+    on this package's path; timed with CUDA events after one warm-up call."""
+    import torch.nn.functional as F
+
+    w = ctx[0]
+    dev = torch.device("cuda", local)
+    Hq, n, d = w.q.shape
+    q, k, v = w.q[None], w.k[None], w.v[None]
+    stream = torch.cuda.current_stream(dev)
+    F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 2
+    e0.record(stream)
+    for _ in range(reps):
+        F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    dense_flops = 4.0 * d * Hq * n * (n + 1) / 2
+    return {"impl": "torch SDPA, causal, GQA", "ms": round(ms, 3),
+            "tflops": round(dense_flops / (ms * 1e-3) / 1e12, 1),
+            "speedup_of_sparse_attention": round(ms / attn_flops_ms, 3)}
+
+
 def run_decode(args, local):
     import dynamic_sparse_attention_03_b200 as dsa
 
@@ -486,6 +513,7 @@ def main():
     ap.add_argument("--no-vs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -500,6 +528,8 @@ def main():
     res, ctx = run_ours(args, rank, world, local)
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, ctx, local)
+    if not args.no_dense:
+        res["dense_comparator"] = run_dense(args, ctx, local, res["breakdown_ms"]["attention"])
     if not args.no_decode:
         res["decode"] = run_decode(args, local)
     if not args.no_vs:
