@@ -18,8 +18,9 @@
 //    swizzle, no multicast) for blocks, 16-byte gathers for columns.  A K stage
 //    is refilled once both QK^T products have read it, a V stage once both PV
 //    products have.
-//  * Warp 1 (one thread) issues tcgen05.mma in the order QK_A(t+1), PV_B(t),
-//    QK_B(t+1), PV_A(t+1), ...: S = Q K^T (M=128, N=128, K=d, shared-memory
+//  * Warp 1 walks the MMA schedule warp-uniformly (one elected lane issues),
+//    in the order QK_A(t+1), PV_B(t), QK_B(t+1), PV_A(t+1), ...:
+//    S = Q K^T (M=128, N=128, K=d, shared-memory
 //    operands) into TMEM S_A / S_B, and O += P V (M=128, N=d, K=128) with P
 //    read from TMEM (aliased onto the first 64 columns of S) and V from shared
 //    memory.  tcgen05.mma operations of a CTA run in issue order, so the PV
@@ -348,73 +349,88 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_pv = umma_idesc_bf16(128, D, 1);
-      bool ok = mbar_wait(bar(AB_Q), 0, ab);
-      auto qk = [&](int tile, int ks, int nsl) {
-        const uint32_t idesc_qk = umma_idesc_bf16(128, nsl * 64, 0);
-        const uint32_t dS = tmem + kTmemS + 128u * (uint32_t)tile;
+    // The whole warp walks the schedule, so every descriptor and TMEM address
+    // is warp-uniform and computed once per tile from fixed bases (a
+    // descriptor's start field is the shared address >> 4; adding an offset
+    // >> 4 moves it, with no carry past the 14-bit field below 256 KB).  One
+    // elected lane issues each tcgen05 instruction.
+    const bool issuer = elect_one();
+    const uint32_t idesc_pv = umma_idesc_bf16(128, D, 1);
+    const uint32_t idesc_qk2 = umma_idesc_bf16(128, 128, 0), idesc_qk1 = umma_idesc_bf16(128, 64, 0);
+    const uint64_t dQ0 = umma_desc_sw128(sQ(0), 16, 1024), dQ1 = umma_desc_sw128(sQ(1), 16, 1024);
+    const uint64_t dK0 = umma_desc_sw128(sK(0), 16, 1024);
+    const uint64_t dV0 = umma_desc_sw128(sV(0), Lay::kHalf, 1024);
+    auto qk = [&](int tile, int ks, int nsl) {
+      const uint32_t idesc = nsl > 1 ? idesc_qk2 : idesc_qk1;
+      const uint32_t dS = tmem + kTmemS + 128u * (uint32_t)tile;
+      const uint64_t a0 = tile ? dQ1 : dQ0;
+      const uint64_t b0 = dK0 + (uint64_t)(((uint32_t)ks * (uint32_t)Lay::kTile) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = umma_desc_sw128(sQ(tile) + (kk >> 2) * Lay::kHalf + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = umma_desc_sw128(sK(ks) + (kk >> 2) * Lay::kHalf + (kk & 3) * 32, 16, 1024);
-          umma_bf16_ss(dS, a, b, idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar(AB_SFULL + tile));
-      };
-      auto pv = [&](int tile, int u, int nsl) {
-        const uint32_t vst = sV(u % kAttnVS);
-        const uint32_t pa = tmem + kTmemS + 128u * (uint32_t)tile;   // P aliases the first 64 columns of S
-        for (int kk = 0; kk < nsl * 4; ++kk) {
-          const uint64_t b = umma_desc_sw128(vst + kk * 2048, Lay::kHalf, 1024);
-          umma_bf16_ts(tmem + kTmemO + 128u * (uint32_t)tile, pa + 8u * (uint32_t)kk, b, idesc_pv,
-                       (u > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(bar(AB_PVDONE + tile));
-      };
-      int t = 0;
-      int nsl = 0, last = 1;
-      if (ok) ok = mbar_wait(bar(AB_KFULL), 0, ab);
-      if (ok) {
-        nsl = meta[0].nslots;
-        last = meta[0].last;
-        if (nsl > 0) {
-          tc_fence_after();
-          qk(0, 0, nsl);
-          if (hasB) qk(1, 0, nsl);
-          umma_commit(bar(AB_KEMPTY));
-        }
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * Lay::kHalf + (kk & 3) * 32) >> 4);
+        if (issuer) umma_bf16_ss(dS, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
       }
-      while (ok && nsl > 0) {
-        int nsl_next = 0, last_next = 1;
-        // PV_A(t) ; QK_A(t+1)
-        if (!mbar_wait(bar(AB_PFULL + 0), t & 1, ab)) { ok = false; break; }
-        if (!mbar_wait(bar(AB_VFULL + (t % kAttnVS)), (t / kAttnVS) & 1, ab)) { ok = false; break; }
+      if (issuer) umma_commit(bar(AB_SFULL + tile));
+    };
+    auto pv = [&](int tile, int u, int nsl) {
+      const uint64_t b0 = dV0 + (uint64_t)(((uint32_t)(u % kAttnVS) * (uint32_t)Lay::kTile) >> 4);
+      const uint32_t pa = tmem + kTmemS + 128u * (uint32_t)tile;   // P aliases the first 64 columns of S
+      const uint32_t dO = tmem + kTmemO + 128u * (uint32_t)tile;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        if (kk < nsl * 4 && issuer)
+          umma_bf16_ts(dO, pa + 8u * (uint32_t)kk, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                       (u > 0 || kk > 0) ? 1u : 0u);
+      }
+      if (issuer) umma_commit(bar(AB_PVDONE + tile));
+    };
+    bool ok = mbar_wait_warp(bar(AB_Q), 0, ab);
+    int t = 0;
+    int nsl = 0, last = 1;
+    if (ok) ok = mbar_wait_warp(bar(AB_KFULL), 0, ab);
+    if (ok) {
+      nsl = meta[0].nslots;
+      last = meta[0].last;
+      if (nsl > 0) {
         tc_fence_after();
-        pv(0, t, nsl);
-        if (!last) {
-          const int ks = (t + 1) % kAttnKS;
-          if (!mbar_wait(bar(AB_KFULL + ks), ((t + 1) / kAttnKS) & 1, ab)) { ok = false; break; }
-          nsl_next = meta[(t + 1) % kAttnMR].nslots;
-          last_next = meta[(t + 1) % kAttnMR].last;
-          tc_fence_after();
-          qk(0, ks, nsl_next);
-        }
-        // PV_B(t) ; QK_B(t+1)
-        if (hasB) {
-          if (!mbar_wait(bar(AB_PFULL + 1), t & 1, ab)) { ok = false; break; }
-          tc_fence_after();
-          pv(1, t, nsl);
-          if (!last) qk(1, (t + 1) % kAttnKS, nsl_next);
-        }
+        qk(0, 0, nsl);
+        if (hasB) qk(1, 0, nsl);
+        if (issuer) umma_commit(bar(AB_KEMPTY));
+      }
+    }
+    while (ok && nsl > 0) {
+      int nsl_next = 0, last_next = 1;
+      // PV_A(t) ; QK_A(t+1)
+      if (!mbar_wait_warp(bar(AB_PFULL + 0), t & 1, ab)) { ok = false; break; }
+      if (!mbar_wait_warp(bar(AB_VFULL + (t % kAttnVS)), (t / kAttnVS) & 1, ab)) { ok = false; break; }
+      tc_fence_after();
+      pv(0, t, nsl);
+      if (!last) {
+        const int ks = (t + 1) % kAttnKS;
+        if (!mbar_wait_warp(bar(AB_KFULL + ks), ((t + 1) / kAttnKS) & 1, ab)) { ok = false; break; }
+        nsl_next = meta[(t + 1) % kAttnMR].nslots;
+        last_next = meta[(t + 1) % kAttnMR].last;
+        tc_fence_after();
+        qk(0, ks, nsl_next);
+      }
+      // PV_B(t) ; QK_B(t+1)
+      if (hasB) {
+        if (!mbar_wait_warp(bar(AB_PFULL + 1), t & 1, ab)) { ok = false; break; }
+        tc_fence_after();
+        pv(1, t, nsl);
+        if (!last) qk(1, (t + 1) % kAttnKS, nsl_next);
+      }
+      if (issuer) {
         umma_commit(bar(AB_VEMPTY + (t % kAttnVS)));
         if (!last) umma_commit(bar(AB_KEMPTY + ((t + 1) % kAttnKS)));
-        if (last) break;
-        nsl = nsl_next;
-        last = last_next;
-        ++t;
       }
-      // Drain: every MMA of this CTA has completed before TMEM is freed.
+      if (last) break;
+      nsl = nsl_next;
+      last = last_next;
+      ++t;
+    }
+    // Drain: every MMA of this CTA has completed before TMEM is freed.
+    if (issuer) {
       umma_commit(bar(AB_DRAIN));
       mbar_wait_cleanup(bar(AB_DRAIN), 0, 200000000ull);
     }
