@@ -473,41 +473,57 @@ __global__ void __launch_bounds__(384, 1)
       const bool fast1 = __all_sync(0xFFFFFFFFu, none1 || vm1 == ~0ull);
       if (!mbar_wait_warp(bar(AB_SFULL + tile), t & 1, ab)) { ok = false; break; }
       tc_fence_after();
-      // pass 1: row max of the raw scores (the scale is positive, so it commutes)
-      float mx = -INFINITY;
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        if (sl >= nsl) break;
-        uint32_t ra[32], rb[32];
-        tmem_ld32(sS + 64 * sl, ra);
-        tmem_ld32(sS + 64 * sl + 32, rb);
-        tmem_wait_ld();
-        reg_fence(ra);
-        reg_fence(rb);
-        const unsigned long long vm = sl ? vm1 : vm0;
-        float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
-        if (sl ? fast1 : fast0) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            c0 = fmaxf(c0, __uint_as_float(ra[c]));
-            c1 = fmaxf(c1, __uint_as_float(ra[c + 1]));
-            c2 = fmaxf(c2, __uint_as_float(rb[c]));
-            c3 = fmaxf(c3, __uint_as_float(rb[c + 1]));
-          }
-          if (sl ? none1 : none0) c0 = c1 = c2 = c3 = -INFINITY;
-        } else {
-          const uint32_t lo = (uint32_t)vm, hi = (uint32_t)(vm >> 32);
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            c0 = fmaxf(c0, ((lo >> c) & 1u) ? __uint_as_float(ra[c]) : -INFINITY);
-            c1 = fmaxf(c1, ((lo >> (c + 1)) & 1u) ? __uint_as_float(ra[c + 1]) : -INFINITY);
-            c2 = fmaxf(c2, ((hi >> c) & 1u) ? __uint_as_float(rb[c]) : -INFINITY);
-            c3 = fmaxf(c3, ((hi >> (c + 1)) & 1u) ? __uint_as_float(rb[c + 1]) : -INFINITY);
-          }
-        }
-        mx = fmaxf(mx, fmaxf(fmaxf(c0, c1), fmaxf(c2, c3)));
+      // The S row of both slots (128 keys) in registers with one TMEM round
+      // trip; hidden keys of partially visible slots are set to -inf first.
+      uint32_t sv[4][32];
+      tmem_ld32(sS, sv[0]);
+      tmem_ld32(sS + 32, sv[1]);
+      if (nsl > 1) {
+        tmem_ld32(sS + 64, sv[2]);
+        tmem_ld32(sS + 96, sv[3]);
       }
-      const float mt = mx * sl2;
+      tmem_wait_ld();
+      reg_fence(sv[0]);
+      reg_fence(sv[1]);
+      reg_fence(sv[2]);
+      reg_fence(sv[3]);
+      if (!fast0) {
+        const uint32_t lo = (uint32_t)vm0, hi = (uint32_t)(vm0 >> 32);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          sv[0][c] = ((lo >> c) & 1u) ? sv[0][c] : 0xFF800000u;
+          sv[1][c] = ((hi >> c) & 1u) ? sv[1][c] : 0xFF800000u;
+        }
+      }
+      if (nsl > 1 && !fast1) {
+        const uint32_t lo = (uint32_t)vm1, hi = (uint32_t)(vm1 >> 32);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          sv[2][c] = ((lo >> c) & 1u) ? sv[2][c] : 0xFF800000u;
+          sv[3][c] = ((hi >> c) & 1u) ? sv[3][c] : 0xFF800000u;
+        }
+      }
+      // row max of the raw scores over the visible keys (the scale is positive)
+      float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
+      if (!none0) {
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          c0 = fmax3(c0, __uint_as_float(sv[0][c]), __uint_as_float(sv[0][c + 1]));
+          c1 = fmax3(c1, __uint_as_float(sv[0][c + 2]), __uint_as_float(sv[0][c + 3]));
+          c2 = fmax3(c2, __uint_as_float(sv[1][c]), __uint_as_float(sv[1][c + 1]));
+          c3 = fmax3(c3, __uint_as_float(sv[1][c + 2]), __uint_as_float(sv[1][c + 3]));
+        }
+      }
+      if (nsl > 1 && !none1) {
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          c0 = fmax3(c0, __uint_as_float(sv[2][c]), __uint_as_float(sv[2][c + 1]));
+          c1 = fmax3(c1, __uint_as_float(sv[2][c + 2]), __uint_as_float(sv[2][c + 3]));
+          c2 = fmax3(c2, __uint_as_float(sv[3][c]), __uint_as_float(sv[3][c + 1]));
+          c3 = fmax3(c3, __uint_as_float(sv[3][c + 2]), __uint_as_float(sv[3][c + 3]));
+        }
+      }
+      const float mt = fmaxf(fmaxf(c0, c1), fmaxf(c2, c3)) * sl2;
       float m_new = m_run;
       bool rescale = false;
       if (m_run == -INFINITY) {
@@ -518,53 +534,30 @@ __global__ void __launch_bounds__(384, 1)
       }
       const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
       const float nmu = (m_new == -INFINITY) ? 0.f : -m_new;
-      // pass 2: p = 2^(s*scale*log2e - m), P (bf16, two keys per column) over
-      // the first 64 columns of S: chunk 2*h2 and 2*h2+1 are read before the
-      // 32 columns at 32*h2 are written, and those columns were read earlier.
+      // p = 2^(s*scale*log2e - m); P (bf16, two keys per 32-bit column) over the
+      // first 64 columns of S, which have all been read above.
       float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int sl = 0; sl < 2; ++sl) {
         if (sl >= nsl) break;
-        uint32_t ra[32], rb[32];
-        tmem_ld32(sS + 64 * sl, ra);
-        tmem_ld32(sS + 64 * sl + 32, rb);
-        tmem_wait_ld();
-        reg_fence(ra);
-        reg_fence(rb);
         const bool none = sl ? none1 : none0;
-        const float k2 = none ? 0.f : sl2;             // hidden slot: 2^(0*s - inf) = 0
+        // hidden slot: 2^(0*s - inf) = 0 on the fast path; masked keys are
+        // already -inf (and must not be multiplied by 0)
+        const float k2 = (none && (sl ? fast1 : fast0)) ? 0.f : sl2;
         const float b2 = none ? -INFINITY : nmu;
         uint32_t pk[32];
-        if (sl ? fast1 : fast0) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float2 ea = ffma2(make_float2(__uint_as_float(ra[2 * j]), __uint_as_float(ra[2 * j + 1])),
-                                    make_float2(k2, k2), make_float2(b2, b2));
-            const float2 eb = ffma2(make_float2(__uint_as_float(rb[2 * j]), __uint_as_float(rb[2 * j + 1])),
-                                    make_float2(k2, k2), make_float2(b2, b2));
-            const float2 pa = make_float2(ex2_approx(ea.x), ex2_approx(ea.y));
-            const float2 pb = make_float2(ex2_approx(eb.x), ex2_approx(eb.y));
-            sum2 = fadd2(sum2, fadd2(pa, pb));
-            pk[j] = pack_bf16x2(pa.x, pa.y);
-            pk[16 + j] = pack_bf16x2(pb.x, pb.y);
-          }
-        } else {
-          const unsigned long long vm = sl ? vm1 : vm0;
-          const uint32_t lo = (uint32_t)vm, hi = (uint32_t)(vm >> 32);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float a0 = ((lo >> (2 * j)) & 1u) ? __uint_as_float(ra[2 * j]) : -INFINITY;
-            const float a1 = ((lo >> (2 * j + 1)) & 1u) ? __uint_as_float(ra[2 * j + 1]) : -INFINITY;
-            const float b0 = ((hi >> (2 * j)) & 1u) ? __uint_as_float(rb[2 * j]) : -INFINITY;
-            const float b1 = ((hi >> (2 * j + 1)) & 1u) ? __uint_as_float(rb[2 * j + 1]) : -INFINITY;
-            const float2 ea = ffma2(make_float2(a0, a1), make_float2(sl2, sl2), make_float2(nmu, nmu));
-            const float2 eb = ffma2(make_float2(b0, b1), make_float2(sl2, sl2), make_float2(nmu, nmu));
-            const float2 pa = make_float2(ex2_approx(ea.x), ex2_approx(ea.y));
-            const float2 pb = make_float2(ex2_approx(eb.x), ex2_approx(eb.y));
-            sum2 = fadd2(sum2, fadd2(pa, pb));
-            pk[j] = pack_bf16x2(pa.x, pa.y);
-            pk[16 + j] = pack_bf16x2(pb.x, pb.y);
-          }
+        for (int j = 0; j < 16; ++j) {
+          const float2 ea = ffma2(make_float2(__uint_as_float(sv[2 * sl][2 * j]), __uint_as_float(sv[2 * sl][2 * j + 1])),
+                                  make_float2(k2, k2), make_float2(b2, b2));
+          const float2 eb =
+              ffma2(make_float2(__uint_as_float(sv[2 * sl + 1][2 * j]), __uint_as_float(sv[2 * sl + 1][2 * j + 1])),
+                    make_float2(k2, k2), make_float2(b2, b2));
+          const float2 pa = make_float2(ex2_approx(ea.x), ex2_approx(ea.y));
+          const float2 pb = make_float2(ex2_approx(eb.x), ex2_approx(eb.y));
+          sum2 = fadd2(sum2, fadd2(pa, pb));
+          pk[j] = pack_bf16x2(pa.x, pa.y);
+          pk[16 + j] = pack_bf16x2(pb.x, pb.y);
         }
         tmem_st32(sS + 32 * sl, pk);
       }
