@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(AB_SFULL + b), 1);
-      mbar_init(bar(AB_PFULL + b), 128);
+      mbar_init(bar(AB_PFULL + b), 4);   // one arrival per softmax warp
       mbar_init(bar(AB_PVDONE + b), 1);
     }
     for (int m = 0; m < kAttnMR; ++m) mbar_init(bar(AB_META + m), 1);
@@ -400,19 +400,19 @@ __global__ void __launch_bounds__(384, 1)
     }
     while (ok && nsl > 0) {
       int nsl_next = 0, last_next = 1;
-      // PV_A(t) ; QK_A(t+1)
-      if (!mbar_wait_warp(bar(AB_PFULL + 0), t & 1, ab)) { ok = false; break; }
+      // PV_A(t) ; QK_A(t+1).  The operand tiles usually land before P does,
+      // so their waits come first and P_A(t) is consumed as soon as it is ready.
+      const int ks = (t + 1) % kAttnKS;
       if (!mbar_wait_warp(bar(AB_VFULL + (t % kAttnVS)), (t / kAttnVS) & 1, ab)) { ok = false; break; }
-      tc_fence_after();
-      pv(0, t, nsl);
       if (!last) {
-        const int ks = (t + 1) % kAttnKS;
         if (!mbar_wait_warp(bar(AB_KFULL + ks), ((t + 1) / kAttnKS) & 1, ab)) { ok = false; break; }
         nsl_next = meta[(t + 1) % kAttnMR].nslots;
         last_next = meta[(t + 1) % kAttnMR].last;
-        tc_fence_after();
-        qk(0, ks, nsl_next);
       }
+      if (!mbar_wait_warp(bar(AB_PFULL + 0), t & 1, ab)) { ok = false; break; }
+      tc_fence_after();
+      pv(0, t, nsl);
+      if (!last) qk(0, ks, nsl_next);
       // PV_B(t) ; QK_B(t+1)
       if (hasB) {
         if (!mbar_wait_warp(bar(AB_PFULL + 1), t & 1, ab)) { ok = false; break; }
@@ -579,7 +579,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(AB_PFULL + tile));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(AB_PFULL + tile));
       any = true;
       if (last) break;
       ++t;
