@@ -284,16 +284,7 @@ __global__ void __launch_bounds__(WARPS * 32) block_select_warp_kernel(const flo
   int need = 0;
   if (!all && !none) {
     const float* src = S + ((size_t)hl * nQB + i) * nQB + 1;
-    uint32_t tmin = 255u, tmax = 0u;   // range of the top key byte (sign and high exponent bits)
-    for (int j = lane; j < L; j += 32) {
-      const float v = src[j];
-      row[j] = v;
-      const uint32_t t = float_key(v) >> 24;
-      tmin = min(tmin, t);
-      tmax = max(tmax, t);
-    }
-    tmin = __reduce_min_sync(0xFFFFFFFFu, tmin);
-    tmax = __reduce_max_sync(0xFFFFFFFFu, tmax);
+    for (int j = lane; j < L; j += 32) row[j] = src[j];
     __syncwarp();
     uint32_t prefix = 0, mask = 0;
     int rem = e;
@@ -301,25 +292,9 @@ __global__ void __launch_bounds__(WARPS * 32) block_select_warp_kernel(const flo
 #pragma unroll
       for (int a = 0; a < 8; ++a) hist[w][lane * 8 + a] = 0u;
       __syncwarp();
-      if (shift == 24 && tmax - tmin < 8u) {
-        // scores of one magnitude share a few top bytes: count them in
-        // registers and reduce over the warp instead of contended atomics
-        uint32_t c8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        for (int j = lane; j < L; j += 32) {
-          const uint32_t t = (float_key(row[j]) >> 24) - tmin;
-#pragma unroll
-          for (int a = 0; a < 8; ++a) c8[a] += (t == (uint32_t)a) ? 1u : 0u;
-        }
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          const uint32_t tot = __reduce_add_sync(0xFFFFFFFFu, c8[a]);
-          if (lane == 0 && tmin + a < 256u) hist[w][tmin + a] = tot;
-        }
-      } else {
-        for (int j = lane; j < L; j += 32) {
-          const uint32_t k = float_key(row[j]);
-          if ((k & mask) == prefix) atomicAdd(&hist[w][(k >> shift) & 255u], 1u);
-        }
+      for (int j = lane; j < L; j += 32) {
+        const uint32_t k = float_key(row[j]);
+        if ((k & mask) == prefix) atomicAdd(&hist[w][(k >> shift) & 255u], 1u);
       }
       __syncwarp();
       uint32_t c[8];
