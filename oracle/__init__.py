@@ -11,7 +11,9 @@ library computes, written from the pages' description of the method:
   slash lines run as 64x64 blocks, vertical lines as 1x64 column tiles.
 * Squeezed Attention ("Squeezed Attention：基于语义聚类的长上下文LLM推理加速"),
   section "技术方案" (online stage): score the query against every cluster
-  centroid, keep the top clusters, attend only over their keys and values.
+  centroid, keep the top clusters, attend only over their keys and values;
+  (offline stage, ``clusters.py``): Lloyd's K-means over the fixed context's
+  keys, the centroids and the cluster -> key map.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg may import this package.  The CUDA product path never calls it, and it
@@ -39,3 +41,14 @@ from .attention import sparse_attention_rows, sparse_attention, dense_lists  # n
 from .decode import decode_centroids, decode_select, decode_attention, sparse_decode  # noqa: F401
 from .ties import compare_index_sets  # noqa: F401
 from .ashape import a_shape_lists  # noqa: F401
+from .clusters import (  # noqa: F401
+    segment_means,
+    kmeans_assign,
+    kmeans_update,
+    kmeans,
+    kmeans_objective,
+    cluster_csr,
+    cluster_select,
+    cluster_tokens,
+    cluster_decode_attention,
+)

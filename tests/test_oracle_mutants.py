@@ -78,3 +78,78 @@ def test_planted_mistake_is_caught(case, monkeypatch):
     for chk in checks:
         with pytest.raises(AssertionError):
             chk()
+
+
+# ---------------------------------------------------------------- K-means clusters
+
+import tests.test_oracle_kmeans as kpins  # noqa: E402
+from oracle import clusters as ocl  # noqa: E402
+
+
+def _assign_no_cnorm(keys, cent):
+    return np.argmin(-2.0 * (keys @ cent.T), axis=1).astype(np.int64)
+
+
+def _assign_argmax(keys, cent):
+    d2 = (keys * keys).sum(axis=1)[:, None] + (cent * cent).sum(axis=1)[None, :] - 2.0 * (keys @ cent.T)
+    return np.argmax(d2, axis=1).astype(np.int64)
+
+
+def _update_sum(keys, assign, cent):
+    out = np.zeros_like(cent)
+    np.add.at(out, assign, keys)
+    return out
+
+
+def _update_empty_zero(keys, assign, cent):
+    C = cent.shape[0]
+    sums = np.zeros_like(cent)
+    np.add.at(sums, assign, keys)
+    cnt = np.maximum(np.bincount(assign, minlength=C), 1).astype(np.float64)
+    return sums / cnt[:, None]
+
+
+def _csr_descending(assign, C):
+    off, tok = ocl.__dict__["_orig_csr"](assign, C)
+    tok = tok.copy()
+    for c in range(C):
+        tok[off[c]:off[c + 1]] = tok[off[c]:off[c + 1]][::-1]
+    return off, tok
+
+
+def _tokens_no_tail(clusters, off, tok, n_ctx, S):
+    parts = [tok[off[c]:off[c + 1]] for c in np.asarray(clusters, dtype=np.int64)]
+    return np.sort(np.concatenate(parts)) if parts else np.zeros(0, dtype=np.int64)
+
+
+@pytest.mark.parametrize("case", ["no_cnorm", "argmax", "update_sum", "empty_zero", "csr_desc", "high_tie", "no_tail"])
+def test_planted_kmeans_mistake_is_caught(case, monkeypatch):
+    def patch(name, fn):
+        monkeypatch.setattr(ocl, name, fn)
+        monkeypatch.setattr(oracle, name, fn)
+
+    if case == "no_cnorm":
+        patch("kmeans_assign", _assign_no_cnorm)
+        checks = [kpins.test_assign_matches_explicit_distance_bruteforce]
+    elif case == "argmax":
+        patch("kmeans_assign", _assign_argmax)
+        checks = [kpins.test_assign_matches_explicit_distance_bruteforce, kpins.test_hand_worked_example]
+    elif case == "update_sum":
+        patch("kmeans_update", _update_sum)
+        checks = [kpins.test_update_is_the_member_mean_and_keeps_empty_clusters, kpins.test_one_cluster_is_the_global_mean]
+    elif case == "empty_zero":
+        patch("kmeans_update", _update_empty_zero)
+        checks = [kpins.test_update_is_the_member_mean_and_keeps_empty_clusters]
+    elif case == "csr_desc":
+        monkeypatch.setitem(ocl.__dict__, "_orig_csr", ocl.cluster_csr)
+        patch("cluster_csr", _csr_descending)
+        checks = [kpins.test_csr_is_a_stable_partition]
+    elif case == "high_tie":
+        monkeypatch.setattr(ocl, "select_top", _high_tie_select)
+        checks = [kpins.test_zero_query_is_the_mean_over_kept_tokens]
+    else:
+        patch("cluster_tokens", _tokens_no_tail)
+        checks = [kpins.test_keep_all_clusters_equals_dense_single_query_attention]
+    for chk in checks:
+        with pytest.raises(AssertionError):
+            chk()
