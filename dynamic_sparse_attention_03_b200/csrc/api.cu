@@ -14,6 +14,7 @@
 #include "../../include/dsa.h"
 #include "ashape.cuh"
 #include "attn_fwd.cuh"
+#include "block_topk.cuh"
 #include "decode.cuh"
 #include "index_kernels.cuh"
 #include "vs_kernels.cuh"
@@ -23,8 +24,8 @@ using namespace dsa;
 namespace {
 
 constexpr size_t kStatusBytes = 256;
-constexpr size_t kScoreChunkBytes = size_t(1) << 30;   // pooled-score scratch per head chunk
 constexpr int kMaxN = 1 << 21;
+constexpr int kTopkMaxGrid = 1024;   // persistent top-k grid: one CTA per SM, at most this many
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -220,7 +221,6 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   const int nQB = n / 64;
   const bool pool_only = (q == nullptr);
   int64_t ppm = 0;
-  int chunk = 0;
   if (pool_only) {
     if (!pooled_k) return DSA_ERR_INVALID_ARG;
   } else {
@@ -230,8 +230,6 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
     if (fixed == ratio || !(keep_ratio == keep_ratio) || keep_ratio > 1.0f) return DSA_ERR_INVALID_ARG;
     if (ratio) ppm = (int64_t)std::floor((double)keep_ratio * 1e6 + 0.5);
     if (max_count(nQB, fixed ? k_fixed : 0, ppm) > kcap) return DSA_ERR_CAPACITY;
-    const size_t per_head = (size_t)nQB * nQB * 4;
-    chunk = (int)std::max<size_t>(1, std::min<size_t>((size_t)Hq, kScoreChunkBytes / per_head));
   }
   WsCarve c(ws);
   uint32_t* status = static_cast<uint32_t*>(c.take(kStatusBytes));
@@ -241,7 +239,12 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   float* k_hi = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hkv * nQB * d * 4));
   float* k_lo = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hkv * nQB * d * 4));
   float* kbar = pooled_k;
-  float* scores = pool_only ? nullptr : static_cast<float*>(c.take((size_t)chunk * nQB * nQB * 4));
+  // kept-column bit masks written by the fused score/top-k kernel and read by
+  // the list kernel: 16 bytes per (head, query block, key chunk of its tile)
+  const int nrt = (nQB + 127) / 128;
+  uint32_t* masks = pool_only ? nullptr
+                              : static_cast<uint32_t*>(c.take((size_t)Hq * topk_mask_words_per_head(nrt) * 4));
+  int* next_tile = pool_only ? nullptr : static_cast<int*>(c.take(sizeof(int)));
   if (!ws) {
     *ws_bytes = c.off;
     return DSA_OK;
@@ -258,45 +261,43 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   if (d == 128) pool_blocks_kernel<128><<<(unsigned)nqb, 256, 0, st>>>(qp, nullptr, nqb, q_hi, q_lo);
   else pool_blocks_kernel<64><<<(unsigned)nqb, 256, 0, st>>>(qp, nullptr, nqb, q_hi, q_lo);
   if (int rc = launch_check()) return rc;
+  // pooled scores and the per-row top-k in one kernel (the scores stay on chip)
   CUtensorMap tqh, tql, tkh, tkl;
   if (!make_tmap_f32(&tqh, q_hi, nqb, d, 128) || !make_tmap_f32(&tql, q_lo, nqb, d, 128) ||
-      !make_tmap_f32(&tkh, k_hi, nkb, d, 64) || !make_tmap_f32(&tkl, k_lo, nkb, d, 64))
+      !make_tmap_f32(&tkh, k_hi, nkb, d, 128) || !make_tmap_f32(&tkl, k_lo, nkb, d, 128))
     return DSA_ERR_CUDA;
-  const int nrt = (nQB + 127) / 128;   // row tiles of 128 query blocks; row tile r has 2r+2 column tiles of 64
-  const unsigned ntiles = (unsigned)(nrt * (nrt + 1));
-  constexpr int kSelWarps = 4;
-  const bool warp_select = nQB <= 4096;   // a row per warp in shared memory
-  const size_t sel_smem = warp_select ? (size_t)kSelWarps * nQB * 4 : (size_t)nQB * 4;
-  int rc = (d == 128) ? set_smem(block_scores_tc_kernel<128>, ScoreTcLayout<128>::kSmemAlloc)
-                      : set_smem(block_scores_tc_kernel<64>, ScoreTcLayout<64>::kSmemAlloc);
-  if (rc) return rc;
-  if (warp_select) {
-    if ((rc = set_smem(block_select_warp_kernel<kSelWarps>, sel_smem))) return rc;
-  } else if ((rc = set_smem(block_select_kernel<256>, sel_smem))) {
-    return rc;
+  TopkParams tp{};
+  tp.block_idx = block_idx;
+  tp.block_cnt = block_cnt;
+  tp.status = status;
+  tp.nQB = nQB;
+  tp.Hq = Hq;
+  tp.grp = Hq / Hkv;
+  tp.kcap = kcap;
+  tp.k_fixed = k_fixed > 0 ? k_fixed : 0;
+  tp.nrt = nrt;
+  tp.ntiles = nrt * Hq;
+  tp.masks = masks;
+  tp.next_tile = next_tile;
+  tp.ppm = ppm;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
+    return DSA_ERR_CUDA;
+  const unsigned grid = (unsigned)std::min(std::min(nsm, kTopkMaxGrid), tp.ntiles);
+  if (cudaMemsetAsync(next_tile, 0, sizeof(int), st) != cudaSuccess) return DSA_ERR_CUDA;
+  int rc;
+  if (d == 128) {
+    if ((rc = set_smem(block_topk_kernel<128>, TopkLayout<128>::kSmemAlloc))) return rc;
+    block_topk_kernel<128><<<grid, 320, TopkLayout<128>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, tp);
+  } else {
+    if ((rc = set_smem(block_topk_kernel<64>, TopkLayout<64>::kSmemAlloc))) return rc;
+    block_topk_kernel<64><<<grid, 320, TopkLayout<64>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, tp);
   }
-  const int grp = Hq / Hkv;
-  const int kf = k_fixed > 0 ? k_fixed : 0;
-  for (int h0 = 0; h0 < Hq; h0 += chunk) {
-    const int hc = std::min(chunk, Hq - h0);
-    dim3 gs(ntiles, hc);
-    if (d == 128)
-      block_scores_tc_kernel<128><<<gs, 128, ScoreTcLayout<128>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, scores, nQB, h0,
-                                                                                   grp, status);
-    else
-      block_scores_tc_kernel<64><<<gs, 128, ScoreTcLayout<64>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, scores, nQB, h0,
-                                                                                 grp, status);
-    if ((rc = launch_check())) return rc;
-    if (warp_select) {
-      const int nrows = hc * nQB;
-      block_select_warp_kernel<kSelWarps><<<(nrows + kSelWarps - 1) / kSelWarps, kSelWarps * 32, sel_smem, st>>>(
-          scores, nQB, h0, nrows, kf, ppm, block_idx, block_cnt, kcap);
-    } else {
-      block_select_kernel<256><<<dim3(nQB, hc), 256, sel_smem, st>>>(scores, nQB, h0, kf, ppm, block_idx, block_cnt,
-                                                                     kcap);
-    }
-    if ((rc = launch_check())) return rc;
-  }
+  if ((rc = launch_check())) return rc;
+  const int64_t nrows = (int64_t)Hq * nQB;
+  block_list_kernel<<<(unsigned)((nrows + 7) / 8), 256, 0, st>>>(tp);
+  if ((rc = launch_check())) return rc;
   return DSA_OK;
 }
 
