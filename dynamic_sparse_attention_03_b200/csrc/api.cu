@@ -44,6 +44,7 @@ struct WsCarve {
 
 int cuda_err(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
 
+
 int launch_check() { return cuda_err(cudaGetLastError()); }
 
 // Dynamic shared memory above 48 KB needs an opt-in per kernel.
@@ -258,10 +259,6 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   if (int rc = launch_check()) return rc;
   if (pool_only) return DSA_OK;
   const auto* qp = static_cast<const __nv_bfloat16*>(q);
-  if (d == 128) pool_blocks_kernel<128><<<(unsigned)nqb, 256, 0, st>>>(qp, nullptr, nqb, q_hi, q_lo);
-  else pool_blocks_kernel<64><<<(unsigned)nqb, 256, 0, st>>>(qp, nullptr, nqb, q_hi, q_lo);
-  if (int rc = launch_check()) return rc;
-  // pooled scores and the per-row top-k in one kernel (the scores stay on chip)
   CUtensorMap tqh, tql, tkh, tkl;
   if (!make_tmap_f32(&tqh, q_hi, nqb, d, 128) || !make_tmap_f32(&tql, q_lo, nqb, d, 128) ||
       !make_tmap_f32(&tkh, k_hi, nkb, d, 128) || !make_tmap_f32(&tkl, k_lo, nkb, d, 128))
@@ -276,27 +273,36 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   tp.kcap = kcap;
   tp.k_fixed = k_fixed > 0 ? k_fixed : 0;
   tp.nrt = nrt;
-  tp.ntiles = nrt * Hq;
   tp.masks = masks;
-  tp.next_tile = next_tile;
   tp.ppm = ppm;
   int dev = 0, nsm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
     return DSA_ERR_CUDA;
+  int rc;
+  if ((rc = (d == 128) ? set_smem(block_topk_kernel<128>, TopkLayout<128>::kSmemAlloc)
+                       : set_smem(block_topk_kernel<64>, TopkLayout<64>::kSmemAlloc)))
+    return rc;
+  if (d == 128) pool_blocks_kernel<128><<<(unsigned)nqb, 256, 0, st>>>(qp, nullptr, nqb, q_hi, q_lo);
+  else pool_blocks_kernel<64><<<(unsigned)nqb, 256, 0, st>>>(qp, nullptr, nqb, q_hi, q_lo);
+  if ((rc = launch_check())) return rc;
+  // pooled scores and the per-row top-k in one kernel (the scores stay on chip)
+  tp.h0 = 0;
+  tp.nh = Hq;
+  tp.ntiles = nrt * Hq;
+  tp.next_tile = next_tile;
   const unsigned grid = (unsigned)std::min(std::min(nsm, kTopkMaxGrid), tp.ntiles);
   if (cudaMemsetAsync(next_tile, 0, sizeof(int), st) != cudaSuccess) return DSA_ERR_CUDA;
-  int rc;
-  if (d == 128) {
-    if ((rc = set_smem(block_topk_kernel<128>, TopkLayout<128>::kSmemAlloc))) return rc;
-    block_topk_kernel<128><<<grid, 320, TopkLayout<128>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, tp);
-  } else {
-    if ((rc = set_smem(block_topk_kernel<64>, TopkLayout<64>::kSmemAlloc))) return rc;
-    block_topk_kernel<64><<<grid, 320, TopkLayout<64>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, tp);
-  }
+  if (d == 128) block_topk_kernel<128><<<grid, 320, TopkLayout<128>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, tp);
+  else block_topk_kernel<64><<<grid, 320, TopkLayout<64>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, tp);
   if ((rc = launch_check())) return rc;
   const int64_t nrows = (int64_t)Hq * nQB;
-  block_list_kernel<<<(unsigned)((nrows + 7) / 8), 256, 0, st>>>(tp);
+  // rows of the last row tile have 4 nrt mask words: 32-word batches
+  const int nbmax = (4 * nrt + 31) / 32;
+  const int64_t list_ctas = std::min<int64_t>((nrows + 7) / 8, (int64_t)nsm * 7);
+  if (nbmax <= 2) block_list_kernel<2><<<(unsigned)list_ctas, 256, 0, st>>>(tp);
+  else if (nbmax <= 8) block_list_kernel<8><<<(unsigned)list_ctas, 256, 0, st>>>(tp);
+  else block_list_kernel<32><<<(unsigned)list_ctas, 256, 0, st>>>(tp);
   if ((rc = launch_check())) return rc;
   return DSA_OK;
 }

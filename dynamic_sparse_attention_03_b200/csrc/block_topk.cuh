@@ -71,6 +71,7 @@ struct TopkParams {
   uint32_t* masks;     // kept-column bits, see topk_mask_row
   int* next_tile;      // tile counter (zero at launch): CTAs take tiles in order, heaviest first
   int nQB, Hq, grp, kcap, k_fixed, nrt, ntiles;
+  int h0, nh;          // q-heads h0 .. h0 + nh - 1 are this launch's (ntiles = nrt * nh)
   int64_t ppm;
 };
 
@@ -122,8 +123,13 @@ struct TopkPub {
   int cnt2[128];   // second thread: nd | nc << 16
 };
 
+// Value bin in [0, 255]: s * inv + nlo clamped to [-1, 256] and rounded to
+// the nearest integer by adding 1.5 * 2^23 (no float-to-int conversion
+// instruction).  Every step is monotone in s, so the bin order is the score
+// order; all passes that compare bins use this same function.
 __device__ __forceinline__ int topk_bin(float s, float inv, float nlo) {
-  int b = __float2int_rd(fmaf(s, inv, nlo));
+  const float x = fminf(fmaxf(fmaf(s, inv, nlo), -1.f), 256.f);
+  const int b = __float_as_int(x + 12582912.f) - 0x4B400000;
   return min(max(b, 0), 255);
 }
 
@@ -142,12 +148,12 @@ __device__ __forceinline__ void hist_clear(const RowWords& W) {
   for (int w = 0; w < 128; ++w) W[w] = 0u;
 }
 
-// Adds 1 to bin b when `on` (else adds 0): a shared-memory reduction, so
-// consecutive adds to one word do not wait on each other's load and store;
-// both threads of a row add into the same words.
+// Adds 1 to bin b when `on` (else adds 0): a shared-memory atomic whose
+// result is unused, so consecutive adds to one word do not wait on each
+// other's load and store; both threads of a row add into the same words.
 __device__ __forceinline__ void hist_add_if(const RowWords& W, int b, bool on) {
   const uint32_t inc = on ? (1u << ((b & 1) << 4)) : 0u;
-  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(W.addr(b >> 1)), "r"(inc) : "memory");
+  atomicAdd(&W[b >> 1], inc);   // result unused: a shared-memory reduction
 }
 
 // Upper-tail quantile of the standard normal: z with P(Z > z) = q, from the
@@ -497,8 +503,8 @@ __global__ void __launch_bounds__(320, 1)
 
   int tcount = 0;
   for (int tile = *tile_slot; tile < p.ntiles && !*abort_flag; tile = *tile_slot, ++tcount) {
-    const int rt = p.nrt - 1 - tile / p.Hq;
-    const int h = tile % p.Hq, g = h / p.grp;
+    const int rt = p.nrt - 1 - tile / p.nh;
+    const int h = p.h0 + tile % p.nh, g = h / p.grp;
     const int nch = rt + 1;   // key chunks of 128 blocks on or before the tile's diagonal
     if (warp == 0) {
       // the tile's Q̄: hi into the per-row region, lo into the first ring stages
@@ -569,11 +575,13 @@ __global__ void __launch_bounds__(320, 1)
     bool more = __syncthreads_or(is_row && pending0) != 0;
     while (more) {
       const bool approx = pass < 2;
+      // the statistics pass reads a sample: every 4th key chunk of long rows
+      const int cstep = (pass == 0 && nch > 4) ? 4 : 1;
       if (warp == 0) {
         // ---------------------------------------------------------- K̄ producer
         bool ok = true;
         if (pass == 0) ok = mbar_wait_warp(qready, (uint32_t)(tcount & 1), ab);   // Q̄ lo left the ring
-        for (int c = 0; c < nch && ok && !*abort_flag; ++c) {
+        for (int c = 0; c < nch && ok && !*abort_flag; c += cstep) {
           if (approx) {
             if (!(ok = claim(spos, GA))) break;
             if (lane == 0) {
@@ -607,7 +615,7 @@ __global__ void __launch_bounds__(320, 1)
           ok = mbar_wait_warp(qready, (uint32_t)(tcount & 1), ab);
           tc_fence_after();
         }
-        for (int c = 0; c < nch && ok; ++c) {
+        for (int c = 0; c < nch && ok; c += cstep) {
           const int sbuf = (int)(chunk_ctr & 1u);
           if (chunk_ctr >= 2u && !(ok = mbar_wait_warp(sempty(sbuf), ((chunk_ctr >> 1) - 1) & 1, ab))) break;
           tc_fence_after();
@@ -664,7 +672,7 @@ __global__ void __launch_bounds__(320, 1)
         else need = 0u;
         const uint32_t wneed = __reduce_or_sync(0xFFFFFFFFu, need);
         const int cbase = second ? kTopkCap : 0;
-        for (int c = 0; c < nch; ++c) {
+        for (int c = 0; c < nch; c += cstep) {
           const int sbuf = (int)(chunk_ctr & 1u);
           if (ok) ok = mbar_wait_warp(sfull(sbuf), (chunk_ctr >> 1) & 1, ab);
           tc_fence_after();
@@ -751,8 +759,8 @@ __global__ void __launch_bounds__(320, 1)
               const float kInf = __int_as_float(0x7f800000);
               if (R.inv > 0.f) {
                 const float lo = -R.nlo / R.inv;
-                R.wlo = (bin == 0) ? -kInf : lo + ((float)bin - 0.25f) / R.inv;
-                R.whi = (bin == 255) ? kInf : lo + ((float)bin + 1.25f) / R.inv;
+                R.wlo = (bin == 0) ? -kInf : lo + ((float)bin - 0.75f) / R.inv;
+                R.whi = (bin == 255) ? kInf : lo + ((float)bin + 0.75f) / R.inv;
               } else {
                 R.wlo = -kInf;
                 R.whi = kInf;
@@ -878,23 +886,41 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
-// Writes the block lists from the masks of block_topk_kernel: one warp per
-// (head, query block), 8 warps per CTA, each with 1024 ids of staging.
+// Writes the block lists from the masks of block_topk_kernel: each warp takes
+// (head, query block) rows in a grid-stride loop, loading the next row's mask
+// words while it writes the current one; 1024 ids of staging per warp.  NB is
+// the number of 32-word mask batches a row can have (rows of row tile rt have
+// 4 (rt + 1) words), so short rows keep few registers and many warps resident.
+template <int NB>
 __global__ void __launch_bounds__(256) block_list_kernel(const TopkParams p) {
   __shared__ int32_t stage_all[8][1024];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * 8 + warp;
-  if (row >= (int64_t)p.Hq * p.nQB) return;
-  const int h = (int)(row / p.nQB), i = (int)(row % p.nQB);
-  const int nwords = ((i >> 7) + 1) * 4, nb = (nwords + 31) / 32;   // nb <= 32 for n <= 2M
-  const uint32_t* mr = topk_mask_row(p.masks, p.nrt, h, i);
-  uint32_t wv[32];
+  const int64_t nrows = (int64_t)p.Hq * p.nQB;
+  const int64_t step = (int64_t)gridDim.x * 8;
+  auto load = [&](int64_t row, uint32_t (&wv)[NB], int& nb) {
+    const int i = (int)(row % p.nQB), h = (int)(row / p.nQB);
+    const int nwords = ((i >> 7) + 1) * 4;
+    nb = (nwords + 31) / 32;
+    const uint32_t* mr = topk_mask_row(p.masks, p.nrt, h, i);
 #pragma unroll
-  for (int b = 0; b < 32; ++b) {
-    const int w = 32 * b + lane;
-    wv[b] = (b < nb && w < nwords) ? __ldcg(mr + w) : 0u;
+    for (int b = 0; b < NB; ++b) {
+      const int w = 32 * b + lane;
+      wv[b] = (b < nb && w < nwords) ? __ldcg(mr + w) : 0u;
+    }
+  };
+  int64_t row = (int64_t)blockIdx.x * 8 + warp;
+  if (row >= nrows) return;
+  uint32_t cur[NB], nxt[NB];
+  int nbc = 0, nbn = 0;
+  load(row, cur, nbc);
+  for (; row < nrows; row += step) {
+    const int64_t nrow = row + step;
+    if (nrow < nrows) load(nrow, nxt, nbn);
+    topk_emit_row<NB>(p, (int)(row / p.nQB), (int)(row % p.nQB), cur, nbc, lane, stage_all[warp]);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) cur[b] = nxt[b];
+    nbc = nbn;
   }
-  topk_emit_row<32>(p, h, i, wv, nb, lane, stage_all[warp]);
 }
 
 }  // namespace dsa
