@@ -12,6 +12,8 @@ Entry points (same names as the C ABI):
   vertical_slash_index   vertical-slash index and its block/column plan
   block_sparse_attn_fwd  causal attention over the chosen blocks and columns
   sparse_decode_attn     centroid-ranked sparse decode
+  kmeans_clusters        K-means key clusters of a fixed context (centroids, cluster -> key map)
+  cluster_decode_attn    decode ranked by K-means cluster centroids
 """
 
 from __future__ import annotations
@@ -27,6 +29,7 @@ import torch
 __all__ = [
     "DSAError", "load_library", "SYMBOLS", "sparse_index_estimate", "pool_keys", "vertical_slash_index",
     "block_sparse_attn_fwd", "sparse_decode_attn", "get_status", "block_index_capacity", "Workspace",
+    "kmeans_clusters", "cluster_decode_attn",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -40,6 +43,8 @@ SYMBOLS = (
     "sparse_decode_attn",
     "sparse_decode_attn_static",
     "a_shape_index",
+    "kmeans_clusters",
+    "cluster_decode_attn",
     "dsa_get_status",
     "dsa_block_index_capacity",
     "dsa_version",
@@ -75,6 +80,8 @@ _SIGS = {
     "sparse_decode_attn": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P, _SZ, _P],
     "sparse_decode_attn_static": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P],
     "a_shape_index": [_I, _I, _I, _I, _P, _P, _I, _P],
+    "kmeans_clusters": [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P],
+    "cluster_decode_attn": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P, _SZ, _P],
     "dsa_get_status": [_P, _P],
     "dsa_block_index_capacity": [_I, _I, _I, _F],
     "dsa_version": [],
@@ -339,3 +346,53 @@ def a_shape_index(Hq: int, n: int, n_sink: int, n_local: int, device=None):
     _check(load_library().a_shape_index(Hq, n, n_sink, n_local, _ptr(bi), _ptr(bc), kcap, _stream(dev)),
            "a_shape_index")
     return bi, bc
+
+
+def kmeans_clusters(k_cache: torch.Tensor, n_ctx: int, n_clusters: int, iters: int,
+                    ws: Optional[Workspace] = None):
+    """Lloyd's K-means over the first n_ctx keys of every (batch, KV head) of
+    k_cache [B][Hkv][S][d] bf16, started from the means of n_clusters equal
+    contiguous segments.  Returns (centroids [B][Hkv][C][d] fp32, assign
+    [B][Hkv][n_ctx] int32, offsets [B][Hkv][C+1] int32, tokens [B][Hkv][n_ctx]
+    int32): the cluster -> key map lists cluster c's keys, ascending, at
+    tokens[offsets[c]:offsets[c+1]]."""
+    _need_cuda(k_cache)
+    _need_dtype(k_cache, torch.bfloat16, "k_cache")
+    B, Hkv, S, d = k_cache.shape
+    dev = k_cache.device
+    C = int(n_clusters)
+    cent = torch.empty((B, Hkv, C, d), dtype=torch.float32, device=dev)
+    assign = torch.empty((B, Hkv, n_ctx), dtype=torch.int32, device=dev)
+    offsets = torch.empty((B, Hkv, C + 1), dtype=torch.int32, device=dev)
+    tokens = torch.empty((B, Hkv, n_ctx), dtype=torch.int32, device=dev)
+    args = [_ptr(k_cache), B, Hkv, S, d, int(n_ctx), C, int(iters), _ptr(cent), _ptr(assign), _ptr(offsets),
+            _ptr(tokens)]
+    _call_with_ws("kmeans_clusters", args, dev, ws)
+    return cent, assign, offsets, tokens
+
+
+def cluster_decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, centroids: torch.Tensor,
+                        offsets: torch.Tensor, tokens: torch.Tensor, n_ctx: int, keep: int,
+                        scale: Optional[float] = None, return_sel: bool = False,
+                        out: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None):
+    """Decode over K-means clusters: q [B][Hq][d], caches [B][Hkv][S][d] bf16,
+    centroids / offsets / tokens from kmeans_clusters.  Each q-head keeps its
+    `keep` best non-empty clusters by q.c (ties to the lower cluster) and attends
+    over their keys plus the unclustered tail [n_ctx, S).  Returns O [B][Hq][d]
+    bf16 (and sel_idx [B][Hq][keep] ascending cluster ids, sel_cnt [B][Hq])."""
+    _need_cuda(q, k_cache, v_cache, centroids, offsets, tokens, out)
+    _need_dtype(centroids, torch.float32, "centroids")
+    B, Hq, d = q.shape
+    Hkv, S = k_cache.shape[1], k_cache.shape[2]
+    C = centroids.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    kcap = max(min(int(keep), C), 1)
+    sel_idx = sel_cnt = None
+    if return_sel:
+        sel_idx = torch.empty((B, Hq, kcap), dtype=torch.int32, device=q.device)
+        sel_cnt = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
+    args = [_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(centroids), _ptr(offsets), _ptr(tokens), B, Hq, Hkv, S, d,
+            int(n_ctx), C, int(keep), float(scale), _ptr(o), _ptr(sel_idx), _ptr(sel_cnt), kcap]
+    _call_with_ws("cluster_decode_attn", args, q.device, ws)
+    return (o, sel_idx, sel_cnt) if return_sel else o

@@ -14,6 +14,7 @@
 #include "../../include/dsa.h"
 #include "ashape.cuh"
 #include "attn_fwd.cuh"
+#include "clusters.cuh"
 #include "block_topk.cuh"
 #include "decode.cuh"
 #include "index_kernels.cuh"
@@ -181,6 +182,16 @@ int launch_decode(const DecodeParams& p, int B, int Hkv, int nchmax, size_t sel_
   if ((rc = launch_check())) return rc;
   if ((rc = set_smem(decode_attn_kernel<D, G>, DecLayout<D>::kBytes))) return rc;
   decode_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 160, DecLayout<D>::kBytes, st>>>(p);
+  return launch_check();
+}
+
+template <int D, int G>
+int launch_cluster_decode(const ClusterParams& cp, int B, int Hkv, int nchmax, size_t sel_smem, cudaStream_t st) {
+  int rc;
+  if ((rc = set_smem(cluster_select_kernel<D, G, 256>, sel_smem))) return rc;
+  cluster_select_kernel<D, G, 256><<<B * Hkv, 256, sel_smem, st>>>(cp);
+  if ((rc = launch_check())) return rc;
+  cluster_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 128, 0, st>>>(cp.dp);
   return launch_check();
 }
 
@@ -505,6 +516,131 @@ int sparse_decode_attn(const void* q, const void* k_cache, const void* v_cache, 
     DSA_DECODE_CASE(1, 64) DSA_DECODE_CASE(2, 64) DSA_DECODE_CASE(4, 64) DSA_DECODE_CASE(8, 64)
     DSA_DECODE_CASE(1, 128) DSA_DECODE_CASE(2, 128) DSA_DECODE_CASE(4, 128) DSA_DECODE_CASE(8, 128)
 #undef DSA_DECODE_CASE
+    default:
+      return DSA_ERR_UNSUPPORTED;
+  }
+  if (rc) return rc;
+  if (d == 128) decode_combine_kernel<128><<<B * Hq, 128, 0, st>>>(p);
+  else decode_combine_kernel<64><<<B * Hq, 128, 0, st>>>(p);
+  return launch_check();
+}
+
+int kmeans_clusters(const void* k_cache, int B, int Hkv, int S, int d, int n_ctx, int C, int iters,
+                    float* centroids, int32_t* assign, int32_t* offsets, int32_t* tokens, void* ws, size_t* ws_bytes,
+                    dsa_stream_t stream) {
+  if (!k_cache || !centroids || !assign || !offsets || !tokens || !ws_bytes) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || S <= 0 || n_ctx <= 0 || n_ctx > S || C <= 0 || iters <= 0) return DSA_ERR_INVALID_ARG;
+  if (C > n_ctx) return DSA_ERR_INVALID_ARG;   // every starting segment holds a key
+  if ((d != 64 && d != 128) || C > kKmMaxC) return DSA_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hkv > 65535 || (int64_t)S * d >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(k_cache) || !aligned16(centroids)) return DSA_ERR_INVALID_ARG;
+  const int BG = B * Hkv;
+  WsCarve c(ws);
+  uint32_t* status = static_cast<uint32_t*>(c.take(kStatusBytes));
+  (void)status;
+  float* cnorm = static_cast<float*>(c.take((size_t)BG * C * 4));
+  if (!ws) {
+    *ws_bytes = c.off;
+    return DSA_OK;
+  }
+  if (*ws_bytes < c.off) return DSA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  KmParams p{};
+  p.k = static_cast<const __nv_bfloat16*>(k_cache);
+  p.cent = centroids;
+  p.cnorm = cnorm;
+  p.assign = assign;
+  p.off = offsets;
+  p.tok = tokens;
+  p.S = S;
+  p.n_ctx = n_ctx;
+  p.C = C;
+  int rc;
+  const dim3 gi(C, BG), ga((n_ctx + 127) / 128, BG), gu((C + 7) / 8, BG);
+  if (d == 128) {
+    if ((rc = set_smem(kmeans_assign_kernel<128>, KmAssignLayout<128>::kBytes))) return rc;
+    kmeans_init_kernel<128><<<gi, 128, 0, st>>>(p);
+  } else {
+    if ((rc = set_smem(kmeans_assign_kernel<64>, KmAssignLayout<64>::kBytes))) return rc;
+    kmeans_init_kernel<64><<<gi, 64, 0, st>>>(p);
+  }
+  if ((rc = launch_check())) return rc;
+  for (int it = 0; it < iters; ++it) {
+    if (d == 128) kmeans_assign_kernel<128><<<ga, 256, KmAssignLayout<128>::kBytes, st>>>(p);
+    else kmeans_assign_kernel<64><<<ga, 256, KmAssignLayout<64>::kBytes, st>>>(p);
+    if ((rc = launch_check())) return rc;
+    kmeans_csr_kernel<<<BG, 1024, 0, st>>>(p);
+    if ((rc = launch_check())) return rc;
+    if (d == 128) kmeans_update_kernel<128><<<gu, 256, 0, st>>>(p);
+    else kmeans_update_kernel<64><<<gu, 256, 0, st>>>(p);
+    if ((rc = launch_check())) return rc;
+  }
+  return DSA_OK;
+}
+
+int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache, const float* centroids,
+                        const int32_t* offsets, const int32_t* tokens, int B, int Hq, int Hkv, int S, int d,
+                        int n_ctx, int C, int keep, float scale, void* o, int32_t* sel_idx, int32_t* sel_cnt, int kcap,
+                        void* ws, size_t* ws_bytes, dsa_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !centroids || !offsets || !tokens || !o || !ws_bytes) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || n_ctx <= 0 || n_ctx > S || C <= 0 || keep < 0)
+    return DSA_ERR_INVALID_ARG;
+  if (keep == 0 && n_ctx == S) return DSA_ERR_INVALID_ARG;   // nothing to attend
+  if ((d != 64 && d != 128) || C > kKmMaxC) return DSA_ERR_UNSUPPORTED;
+  const int grp = Hq / Hkv;
+  if (grp != 1 && grp != 2 && grp != 4 && grp != 8) return DSA_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hkv > 65535 || (int64_t)S * d >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(centroids)) return DSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (sel_idx && kcap < std::min(keep, C)) return DSA_ERR_CAPACITY;
+  const size_t sel_smem = (size_t)grp * d * 4 + (size_t)grp * C * 4 + (size_t)C * 12 + C;
+  if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
+  const int nchmax = (S + kDecChunk - 1) / kDecChunk;
+  WsCarve c(ws);
+  ClusterParams cp{};
+  DecodeParams& p = cp.dp;
+  p.status = static_cast<uint32_t*>(c.take(kStatusBytes));
+  p.uidx = static_cast<int32_t*>(c.take((size_t)B * Hkv * S * 4));
+  p.umask = static_cast<uint8_t*>(c.take((size_t)B * Hkv * S));
+  p.ucnt = static_cast<int32_t*>(c.take((size_t)B * Hkv * 4));
+  p.part_ml = static_cast<float*>(c.take((size_t)B * Hq * nchmax * 2 * 4));
+  p.part_acc = static_cast<float*>(c.take((size_t)B * Hq * nchmax * d * 4));
+  if (!ws) {
+    *ws_bytes = c.off;
+    return DSA_OK;
+  }
+  if (*ws_bytes < c.off) return DSA_ERR_INVALID_ARG;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kc = static_cast<const __nv_bfloat16*>(k_cache);
+  p.vc = static_cast<const __nv_bfloat16*>(v_cache);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.sel_idx = sel_idx;
+  p.sel_cnt = sel_cnt;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.nb = S;
+  p.grp = grp;
+  p.keep = keep;
+  p.kcap = kcap;
+  p.nchmax = nchmax;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cp.cent = centroids;
+  cp.off = offsets;
+  cp.tok = tokens;
+  cp.C = C;
+  cp.n_ctx = n_ctx;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int rc;
+  switch (grp * 1000 + d) {
+#define DSA_CLUSTER_CASE(G, DD)                                                                 \
+  case G * 1000 + DD:                                                                           \
+    rc = launch_cluster_decode<DD, G>(cp, B, Hkv, nchmax, sel_smem, st);                        \
+    break;
+    DSA_CLUSTER_CASE(1, 64) DSA_CLUSTER_CASE(2, 64) DSA_CLUSTER_CASE(4, 64) DSA_CLUSTER_CASE(8, 64)
+    DSA_CLUSTER_CASE(1, 128) DSA_CLUSTER_CASE(2, 128) DSA_CLUSTER_CASE(4, 128) DSA_CLUSTER_CASE(8, 128)
+#undef DSA_CLUSTER_CASE
     default:
       return DSA_ERR_UNSUPPORTED;
   }

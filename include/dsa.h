@@ -197,6 +197,52 @@ int sparse_decode_attn_static(const void* q, const void* k_cache, const void* v_
                               void* o, int32_t* sel_idx, int32_t* sel_cnt, int kcap, dsa_stream_t stream);
 
 /*
+ * kmeans_clusters -- the offline stage of cluster-ranked decode (Squeezed
+ * Attention, technical approach: the fixed context's keys are clustered with
+ * K-means; each cluster gets a centroid and each key an index to its cluster).
+ * Lloyd's algorithm over the first n_ctx keys of every (batch, KV head):
+ * centroids start at the means of C equal contiguous segments
+ * (segment c = keys floor(c n_ctx / C) .. floor((c+1) n_ctx / C) - 1); each of
+ * `iters` rounds assigns every key to its nearest centroid (squared Euclidean
+ * distance in fp32, ties to the lower cluster) and moves every non-empty
+ * cluster's centroid to the mean of its keys (an empty cluster keeps its
+ * centroid).  The outputs are the last round's assignment and the centroids
+ * computed from it.
+ *
+ *  k_cache    [B][Hkv][S][d] bf16 (d in {64, 128}); 1 <= C <= n_ctx <= S, C <= 4096.
+ *  centroids  [B][Hkv][C][d] fp32 out.   assign [B][Hkv][n_ctx] int32 out.
+ *  offsets    [B][Hkv][C+1] int32 out, tokens [B][Hkv][n_ctx] int32 out: the
+ *             keys of cluster c, ascending, are tokens[offsets[c] .. offsets[c+1]).
+ *  iters      >= 1 rounds.
+ * Deterministic: the centroid sums run in token order.
+ */
+int kmeans_clusters(const void* k_cache, int B, int Hkv, int S, int d, int n_ctx, int C, int iters,
+                    float* centroids, int32_t* assign, int32_t* offsets, int32_t* tokens, void* ws,
+                    size_t* ws_bytes, dsa_stream_t stream);
+
+/*
+ * cluster_decode_attn -- the online stage over K-means clusters (Squeezed
+ * Attention, technical approach: compare the query with every centroid, keep
+ * the top clusters, attend only over the keys and values of those clusters).
+ * Each q-head ranks the non-empty clusters of its KV head by the raw score
+ * q.c, keeps the best min(keep, non-empty) (ties to the lower cluster), and
+ * attends over the keys of the kept clusters plus the unclustered tail
+ * [n_ctx, S) (the newest tokens, the current one included).
+ *
+ *  q          [B][Hq][d] bf16.   k_cache, v_cache [B][Hkv][S][d] bf16.
+ *  centroids, offsets, tokens: kmeans_clusters' outputs for the same cache.
+ *  o          [B][Hq][d] bf16 out.
+ *  sel_idx    optional [B][Hq][kcap] int32 out (ascending kept clusters, -1
+ *             padded), sel_cnt optional [B][Hq]; kcap >= min(keep, C).
+ * K and V rows are gathered by token id; the union of a GQA group's kept
+ * clusters is read once for the group.
+ */
+int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache, const float* centroids,
+                        const int32_t* offsets, const int32_t* tokens, int B, int Hq, int Hkv, int S, int d,
+                        int n_ctx, int C, int keep, float scale, void* o, int32_t* sel_idx, int32_t* sel_cnt,
+                        int kcap, void* ws, size_t* ws_bytes, dsa_stream_t stream);
+
+/*
  * dsa_get_status -- synchronize `stream`, read the workspace's device status
  * word, clear it, and return DSA_OK or the first error recorded on the device
  * (DSA_ERR_TIMEOUT for an expired bounded wait, DSA_ERR_INVALID_ARG for a list
