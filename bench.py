@@ -353,6 +353,63 @@ def run_decode(args, local):
             "centroid_build_GB/s": round(cent_gbs, 1), "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": src}
 
 
+def run_cluster_decode(args, local):
+    """Decode over K-means clusters of the same fixed 128K cache (the Squeezed
+    Attention page's offline clustering): 2048 clusters of the first S - 64
+    keys (3 Lloyd rounds, timed once as the offline build), then per step every
+    q-head keeps its 512 best clusters and attends over them plus the newest
+    64 tokens.  GB/s counts the union of a GQA group's kept clusters' K/V rows
+    (each row is read once per (batch, KV head)), the centroids and q / o."""
+    import dynamic_sparse_attention_03_b200 as dsa
+
+    dev = torch.device("cuda", local)
+    dw = synth.make_decode("decode-b16-128k", device=dev)
+    p = dw.params
+    B, Hq, dd = dw.q.shape
+    Hkv, S = dw.k_cache.shape[1], dw.k_cache.shape[2]
+    C, n_ctx, iters, keep = S // 64, S - 64, 3, p["keep"]
+    ws = dsa.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    cent, _, off, tok = dsa.kmeans_clusters(dw.k_cache, n_ctx, C, iters, ws=ws)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    build_ms = b0.elapsed_time(b1)
+    o, si, sc = dsa.cluster_decode_attn(dw.q, dw.k_cache, dw.v_cache, cent, off, tok, n_ctx, keep,
+                                        return_sel=True, ws=ws)
+    torch.cuda.synchronize()
+    grp = Hq // Hkv
+    size = (off[..., 1:] - off[..., :-1]).long()                      # [B][Hkv][C]
+    mask = torch.zeros((B, Hkv, C), dtype=torch.bool, device=dev)
+    for h in range(Hq):
+        idx = si[:, h].long().clamp(min=0)
+        valid = torch.arange(si.shape[-1], device=dev)[None, :] < sc[:, h:h + 1]
+        m2 = torch.zeros((B, C), dtype=torch.long, device=dev)
+        m2.scatter_add_(1, idx * valid, valid.long())
+        mask[:, h // grp] |= m2 > 0
+    union_tokens = int((size * mask).sum().item()) + B * Hkv * (S - n_ctx)
+    total = union_tokens * 2 * dd * 2 + B * Hkv * C * dd * 4 + 2 * B * Hq * dd * 2
+    for _ in range(3):
+        dsa.cluster_decode_attn(dw.q, dw.k_cache, dw.v_cache, cent, off, tok, n_ctx, keep, out=o, ws=ws)
+    torch.cuda.synchronize()
+    reps = 20
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        dsa.cluster_decode_attn(dw.q, dw.k_cache, dw.v_cache, cent, off, tok, n_ctx, keep, out=o, ws=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    peaks, src = load_peaks()
+    gbs = total / (ms * 1e-3) / 1e9
+    del dw
+    return {"workload": "decode-b16-128k, 2048 K-means clusters of the first S-64 keys, keep 512 + tail",
+            "ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+            "bytes_per_step": total, "union_tokens": union_tokens, "kmeans_build_ms": round(build_ms, 2),
+            "kmeans_rounds": iters, "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": src}
+
+
 def run_vs(args, local):
     """Vertical-slash prefill layer at 128K: vertical_slash_index followed by
     block_sparse_attn_fwd over the plan's blocks and column tiles.  Effective
@@ -511,6 +568,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama3-8b-128k-bs10")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-clusters", action="store_true")
     ap.add_argument("--no-vs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -533,6 +591,8 @@ def main():
         res["dense_comparator"] = run_dense(args, ctx, local, res["breakdown_ms"]["attention"])
     if not args.no_decode:
         res["decode"] = run_decode(args, local)
+    if not args.no_clusters:
+        res["cluster_decode"] = run_cluster_decode(args, local)
     if not args.no_vs:
         res["vertical_slash"] = run_vs(args, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -595,7 +595,7 @@ int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache,
   if (sel_idx && kcap < std::min(keep, C)) return DSA_ERR_CAPACITY;
   const size_t sel_smem = (size_t)grp * d * 4 + (size_t)grp * C * 4 + (size_t)C * 12 + C;
   if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
-  const int nchmax = (S + kDecChunk - 1) / kDecChunk;
+  const int nchmax = (S + kClChunk - 1) / kClChunk;
   WsCarve c(ws);
   ClusterParams cp{};
   DecodeParams& p = cp.dp;
@@ -645,8 +645,8 @@ int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache,
       return DSA_ERR_UNSUPPORTED;
   }
   if (rc) return rc;
-  if (d == 128) decode_combine_kernel<128><<<B * Hq, 128, 0, st>>>(p);
-  else decode_combine_kernel<64><<<B * Hq, 128, 0, st>>>(p);
+  if (d == 128) decode_combine_kernel<128, kClChunk><<<B * Hq, 128, 0, st>>>(p);
+  else decode_combine_kernel<64, kClChunk><<<B * Hq, 128, 0, st>>>(p);
   return launch_check();
 }
 

@@ -26,7 +26,7 @@
 //                        group's kept clusters flattened into one token list
 //                        with a per-token head mask, followed by the
 //                        unclustered tail [n_ctx, S) that every head attends.
-//  cluster_attn_kernel:  64 tokens of the union list per CTA: K and V rows
+//  cluster_attn_kernel:  2048 tokens of the union list per CTA: K and V rows
 //                        gathered by token id (16-byte loads, each row read
 //                        once for the whole GQA group), an online softmax per
 //                        head with the token's head mask, one partial per
@@ -416,17 +416,22 @@ __global__ void __launch_bounds__(NT) cluster_select_kernel(const ClusterParams 
 }
 
 // ---------------------------------------------------------------- decode: attention over the union
-// One CTA of 4 warps per (batch x KV head, 64 tokens of the union list):
-// warp w takes tokens 16 w .. 16 w + 15, the two half warps alternate tokens,
-// lane % 16 owns D / 16 dimensions; rows are gathered straight from global
-// memory with 16-byte (8-byte at D = 64) loads.
+// One CTA of 4 warps per (batch x KV head, kClChunk tokens of the union list),
+// walking them SUB = 8 TPL at a time: warp w takes tokens 2 TPL w .. of each
+// step, the two half warps alternate tokens (TPL tokens per lane: 8, or 4 for
+// 8 q-heads per KV head to bound registers), lane % 16 owns D / 16 dims; rows
+// are gathered straight from global memory with 16-byte (8-byte at D = 64)
+// loads, and an online softmax per (lane, head) runs over the whole chunk.
+constexpr int kClChunk = 2048;
+
 template <int D, int GRP>
 __global__ void __launch_bounds__(128) cluster_attn_kernel(const DecodeParams p) {
   __shared__ float red[4][kMaxGrp][D + 2];
   const int bg = blockIdx.x, chunk = blockIdx.y;
   const int cnt = p.ucnt[bg];
-  const int u0 = chunk * kDecChunk;
-  if (u0 >= cnt) return;
+  const int c0 = chunk * kClChunk;
+  if (c0 >= cnt) return;
+  const int c1 = min(cnt, c0 + kClChunk);
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int DPL = D / 16;
@@ -440,83 +445,94 @@ __global__ void __launch_bounds__(128) cluster_attn_kernel(const DecodeParams p)
 #pragma unroll
     for (int a = 0; a < DPL; ++a)
       qv[hh][a] = __bfloat162float(p.q[((size_t)b * p.Hq + g * GRP + hh) * D + dl * DPL + a]) * p.scale_log2;
-  // the 8 tokens of this lane: union positions u0 + 16 w + 2 it + half
-  float kf[8][DPL], vf[8][DPL];
-  uint32_t msk[8];
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int u = u0 + 16 * warp + 2 * it + half;
-    msk[it] = 0u;
-#pragma unroll
-    for (int a = 0; a < DPL; ++a) {
-      kf[it][a] = 0.f;
-      vf[it][a] = 0.f;
-    }
-    if (u < cnt) {
-      msk[it] = um[u];
-      const size_t row = head_base + (size_t)ui[u] * D + dl * DPL;
-      if (DPL == 8) {
-        const uint4 kr = __ldg(reinterpret_cast<const uint4*>(p.kc + row));
-        const uint4 vr = __ldg(reinterpret_cast<const uint4*>(p.vc + row));
-        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
-        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          const float2 kk = __bfloat1622float2(k2[a]), vv = __bfloat1622float2(v2[a]);
-          kf[it][(2 * a) % DPL] = kk.x;
-          kf[it][(2 * a + 1) % DPL] = kk.y;
-          vf[it][(2 * a) % DPL] = vv.x;
-          vf[it][(2 * a + 1) % DPL] = vv.y;
-        }
-      } else {
-        const uint2 kr = __ldg(reinterpret_cast<const uint2*>(p.kc + row));
-        const uint2 vr = __ldg(reinterpret_cast<const uint2*>(p.vc + row));
-        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
-        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
-#pragma unroll
-        for (int a = 0; a < 2; ++a) {
-          const float2 kk = __bfloat1622float2(k2[a]), vv = __bfloat1622float2(v2[a]);
-          kf[it][(2 * a) % DPL] = kk.x;
-          kf[it][(2 * a + 1) % DPL] = kk.y;
-          vf[it][(2 * a) % DPL] = vv.x;
-          vf[it][(2 * a + 1) % DPL] = vv.y;
-        }
-      }
-    }
-  }
   float m[GRP], l[GRP], acc[GRP][DPL];
 #pragma unroll
   for (int hh = 0; hh < GRP; ++hh) {
-    float sc[8];
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      float d0 = 0.f;
-#pragma unroll
-      for (int a = 0; a < DPL; ++a) d0 = fmaf(qv[hh][a], kf[it][a], d0);
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) d0 += __shfl_xor_sync(0xFFFFFFFFu, d0, o);
-      sc[it] = ((msk[it] >> hh) & 1u) ? d0 : -INFINITY;
-    }
-    float mb = sc[0];
-#pragma unroll
-    for (int it = 1; it < 8; ++it) mb = fmaxf(mb, sc[it]);
-    mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 16));
-    m[hh] = mb;
-    float ls = 0.f;
+    m[hh] = -INFINITY;
+    l[hh] = 0.f;
 #pragma unroll
     for (int a = 0; a < DPL; ++a) acc[hh][a] = 0.f;
-    if (mb != -INFINITY) {
+  }
+  constexpr int TPL = GRP >= 8 ? 4 : 8;
+  for (int u0 = c0; u0 < c1; u0 += 8 * TPL) {
+    // this lane's TPL tokens: union positions u0 + 2 TPL w + 2 it + half
+    float kf[TPL][DPL], vf[TPL][DPL];
+    uint32_t msk[TPL];
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const float pe = ex2_approx(sc[it] - mb);   // -inf -> 0
+    for (int it = 0; it < TPL; ++it) {
+      const int u = u0 + 2 * TPL * warp + 2 * it + half;
+      msk[it] = 0u;
+#pragma unroll
+      for (int a = 0; a < DPL; ++a) {
+        kf[it][a] = 0.f;
+        vf[it][a] = 0.f;
+      }
+      if (u < c1) {
+        msk[it] = um[u];
+        const size_t row = head_base + (size_t)ui[u] * D + dl * DPL;
+        if (DPL == 8) {
+          const uint4 kr = __ldg(reinterpret_cast<const uint4*>(p.kc + row));
+          const uint4 vr = __ldg(reinterpret_cast<const uint4*>(p.vc + row));
+          const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+          const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            const float2 kk = __bfloat1622float2(k2[a]), vv = __bfloat1622float2(v2[a]);
+            kf[it][(2 * a) % DPL] = kk.x;
+            kf[it][(2 * a + 1) % DPL] = kk.y;
+            vf[it][(2 * a) % DPL] = vv.x;
+            vf[it][(2 * a + 1) % DPL] = vv.y;
+          }
+        } else {
+          const uint2 kr = __ldg(reinterpret_cast<const uint2*>(p.kc + row));
+          const uint2 vr = __ldg(reinterpret_cast<const uint2*>(p.vc + row));
+          const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+          const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            const float2 kk = __bfloat1622float2(k2[a]), vv = __bfloat1622float2(v2[a]);
+            kf[it][(2 * a) % DPL] = kk.x;
+            kf[it][(2 * a + 1) % DPL] = kk.y;
+            vf[it][(2 * a) % DPL] = vv.x;
+            vf[it][(2 * a + 1) % DPL] = vv.y;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) {
+      float sc[TPL];
+#pragma unroll
+      for (int it = 0; it < TPL; ++it) {
+        float d0 = 0.f;
+#pragma unroll
+        for (int a = 0; a < DPL; ++a) d0 = fmaf(qv[hh][a], kf[it][a], d0);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) d0 += __shfl_xor_sync(0xFFFFFFFFu, d0, o);
+        sc[it] = ((msk[it] >> hh) & 1u) ? d0 : -INFINITY;
+      }
+      float mb = sc[0];
+#pragma unroll
+      for (int it = 1; it < TPL; ++it) mb = fmaxf(mb, sc[it]);
+      mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 16));
+      const float mn = fmaxf(m[hh], mb);
+      if (mn == -INFINITY) continue;   // nothing of this head yet (warp-uniform)
+      const float alpha = ex2_approx(m[hh] - mn);   // m = -inf -> 0
+      float ls = 0.f;
+#pragma unroll
+      for (int a = 0; a < DPL; ++a) acc[hh][a] *= alpha;
+#pragma unroll
+      for (int it = 0; it < TPL; ++it) {
+        const float pe = ex2_approx(sc[it] - mn);   // -inf -> 0
         ls += pe;
 #pragma unroll
         for (int a = 0; a < DPL; ++a) acc[hh][a] = fmaf(pe, vf[it][a], acc[hh][a]);
       }
+      l[hh] = l[hh] * alpha + ls;
+      m[hh] = mn;
     }
-    l[hh] = ls;
   }
-  // merge the half warps (same dims, same max), then the 4 warps
+  // merge the half warps (same dims, same running max), then the 4 warps
 #pragma unroll
   for (int hh = 0; hh < GRP; ++hh) {
     l[hh] += __shfl_xor_sync(0xFFFFFFFFu, l[hh], 16);

@@ -322,11 +322,13 @@ __global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams 
 }
 
 // ---------------------------------------------------------------- combine
-template <int D>
+// CHUNK: union entries per attention CTA (blocks here; tokens for the
+// cluster-ranked decode).
+template <int D, int CHUNK = kDecChunk>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
   const int bh = blockIdx.x;   // b*Hq + h
   const int b = bh / p.Hq, h = bh % p.Hq, g = h / p.grp;
-  const int nch = (p.ucnt[b * p.Hkv + g] + kDecChunk - 1) / kDecChunk;
+  const int nch = (p.ucnt[b * p.Hkv + g] + CHUNK - 1) / CHUNK;
   const float* ml = p.part_ml + (size_t)bh * p.nchmax * 2;
   float M = -INFINITY;
   for (int c = 0; c < nch; ++c) M = fmaxf(M, ml[2 * c]);
