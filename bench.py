@@ -39,6 +39,10 @@ if ROOT not in sys.path:
 
 import synth  # noqa: E402
 
+# DRAM bytes (read + write) of one bsa_fwd_kernel launch, measured with ncu
+# (dram__bytes_read.sum + dram__bytes_write.sum) on this bench's own command
+# for the workload; None for workloads without such a capture.
+BSA_TRAFFIC = {"llama3-8b-128k-bs10": 6.57e9, "llama3-8b-32k-bs10": 7.096e8}
 METRIC = "block-sparse prefill effective TFLOP/s at 128K (selected-block FLOPs)"
 UNIT = "TFLOP/s"
 DIAG_ELEMS = 64 * 65 // 2
@@ -261,7 +265,9 @@ def run_ours(args, rank, world, local):
         "index_reuse": reuse,
         "effective_flops_per_step": flops,
         "roofline": {"bound": "tensor", "kernel": "bsa_fwd_kernel<128>", "achieved": round(achieved, 2),
-                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": BSA_TRAFFIC.get(args.workload),
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch",
                      "peak_source": f"{src} bf16_tflops_sustained"},
         "clocks": clk.summary(),
         "gpu_launches": (launches_per_step * args.steps) if launches_per_step else None,
