@@ -177,6 +177,8 @@ int launch_attn(const void* q, const void* k, const void* v, void* o, int Hq, in
 template <int D, int G>
 int launch_decode(const DecodeParams& p, int B, int Hkv, int nchmax, size_t sel_smem, cudaStream_t st) {
   int rc;
+  decode_score_kernel<D, G><<<dim3(B * Hkv, (p.nb + 63) / 64), 256, 0, st>>>(p);
+  if ((rc = launch_check())) return rc;
   if ((rc = set_smem(decode_select_kernel<D, G, 256>, sel_smem))) return rc;
   decode_select_kernel<D, G, 256><<<B * Hkv, 256, sel_smem, st>>>(p);
   if ((rc = launch_check())) return rc;
@@ -472,7 +474,7 @@ int sparse_decode_attn(const void* q, const void* k_cache, const void* v_cache, 
   const int ncand = force_last ? nb - 1 : nb;
   const int count = std::min(keep, ncand) + force_last;
   if (sel_idx && kcap < count) return DSA_ERR_CAPACITY;
-  const size_t sel_smem = (size_t)grp * d * 4 + (size_t)grp * nb * 4 + (size_t)nb * 4 + nb;
+  const size_t sel_smem = (size_t)grp * nb * 4 + (size_t)nb * 4 + nb;
   if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
   const int nchmax = (nb + kDecChunk - 1) / kDecChunk;
   WsCarve c(ws);
@@ -483,6 +485,7 @@ int sparse_decode_attn(const void* q, const void* k_cache, const void* v_cache, 
   p.ucnt = static_cast<int32_t*>(c.take((size_t)B * Hkv * 4));
   p.part_ml = static_cast<float*>(c.take((size_t)B * Hq * nchmax * 2 * 4));
   p.part_acc = static_cast<float*>(c.take((size_t)B * Hq * nchmax * d * 4));
+  p.scores = static_cast<float*>(c.take((size_t)B * Hq * nb * 4));
   if (!ws) {
     *ws_bytes = c.off;
     return DSA_OK;

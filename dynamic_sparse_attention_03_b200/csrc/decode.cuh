@@ -5,9 +5,12 @@
 // block means (built by the pooling kernel).
 //
 // Kernels:
-//  decode_select_kernel: one CTA per (batch, KV head): q·c for the GQA group's
-//    q-heads, top `keep` per head (ties to the lower block) plus the last
-//    block, and the union of the group's kept blocks with a per-block head mask.
+//  decode_score_kernel: q·c for every (batch, q-head, block), 64 centroid
+//    blocks of one (batch, KV head) per CTA, each centroid row read once for
+//    the group's q-heads.
+//  decode_select_kernel: one CTA per (batch, KV head): top `keep` per q-head of
+//    the group (ties to the lower block) plus the last block, and the union of
+//    the group's kept blocks with a per-block head mask.
 //  decode_attn_kernel: one CTA per (batch, KV head, chunk of union blocks).
 //    One producer thread streams whole 64-token K and V blocks (contiguous
 //    16 KB each at d = 128) into a 4-stage shared-memory ring with bulk copies;
@@ -42,10 +45,63 @@ struct DecodeParams {
   int32_t* ucnt;               // ws [B*Hkv]
   float* part_ml;              // ws [B*Hq][nchmax][2]
   float* part_acc;             // ws [B*Hq][nchmax][D]
+  float* scores;               // ws [B*Hq][nb] q·c
   uint32_t* status;
   int B, Hq, Hkv, S, nb, grp, keep, force_last, kcap, nchmax;
   float scale_log2;
 };
+
+// ---------------------------------------------------------------- scores
+// One CTA of 8 warps per (batch x KV head, 64 centroid blocks): each warp
+// scores 8 blocks for the group's q-heads, loading its 8 rows together.
+template <int D, int GRP>
+__global__ void __launch_bounds__(256) decode_score_kernel(const DecodeParams p) {
+  constexpr int PER = D / 32;
+  const int bg = blockIdx.x, t0 = blockIdx.y * 64;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float qreg[GRP][PER];
+#pragma unroll
+  for (int hh = 0; hh < GRP; ++hh)
+#pragma unroll
+    for (int a = 0; a < PER; ++a)
+      qreg[hh][a] = __bfloat162float(p.q[((size_t)b * p.Hq + g * GRP + hh) * D + lane * PER + a]);
+  const float* crow = p.cent + (size_t)bg * p.nb * D;
+  float cv[8][PER];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int t = t0 + warp * 8 + r;
+    if (t < p.nb) {
+      const float* src = crow + (size_t)t * D + lane * PER;
+      if constexpr (PER == 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(src));
+        cv[r][0] = v.x; cv[r][1] = v.y; cv[r][2] = v.z; cv[r][3] = v.w;
+      } else if constexpr (PER == 2) {
+        const float2 v = __ldg(reinterpret_cast<const float2*>(src));
+        cv[r][0] = v.x; cv[r][1] = v.y;
+      } else {
+#pragma unroll
+        for (int a = 0; a < PER; ++a) cv[r][a] = __ldg(src + a);
+      }
+    } else {
+#pragma unroll
+      for (int a = 0; a < PER; ++a) cv[r][a] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int t = t0 + warp * 8 + r;
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) {
+      float s = 0.f;
+#pragma unroll
+      for (int a = 0; a < PER; ++a) s = fmaf(qreg[hh][a], cv[r][a], s);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+      if (lane == 0 && t < p.nb) p.scores[((size_t)b * p.Hq + g * GRP + hh) * p.nb + t] = s;
+    }
+  }
+}
 
 // ---------------------------------------------------------------- select
 template <int D, int GRP, int NT>
@@ -56,44 +112,12 @@ __global__ void __launch_bounds__(NT) decode_select_kernel(const DecodeParams p)
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int nb = p.nb;
   constexpr int grp = GRP;
-  float* qf = reinterpret_cast<float*>(dsm);                 // [grp][D]
-  float* sc = qf + grp * D;                                   // [grp][nb]
+  float* sc = reinterpret_cast<float*>(dsm);                              // [grp][nb]
   int32_t* tmp = reinterpret_cast<int32_t*>(sc + (size_t)grp * nb);   // [nb]
   uint8_t* mask = reinterpret_cast<uint8_t*>(tmp + nb);      // [nb]
-  for (int x = threadIdx.x; x < grp * D; x += NT) {
-    const int hh = x / D, c = x % D;
-    qf[x] = __bfloat162float(p.q[((size_t)b * p.Hq + g * grp + hh) * D + c]);
-  }
+  const float* gsc = p.scores + ((size_t)b * p.Hq + g * grp) * nb;   // the group's rows are contiguous
+  for (int x = threadIdx.x; x < grp * nb; x += NT) sc[x] = gsc[x];
   for (int x = threadIdx.x; x < nb; x += NT) mask[x] = 0;
-  __syncthreads();
-  // scores: one warp per centroid row, lanes over d
-  constexpr int PER = D / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float qreg[GRP][PER];
-#pragma unroll
-  for (int hh = 0; hh < grp; ++hh)
-#pragma unroll
-    for (int a = 0; a < PER; ++a) qreg[hh][a] = qf[hh * D + lane * PER + a];
-  const float* crow = p.cent + (size_t)bg * nb * D;
-  for (int t = warp; t < nb; t += NT / 32) {
-    float cv[PER];
-    if (PER == 4) {
-      const float4 v4 = __ldg(reinterpret_cast<const float4*>(crow + (size_t)t * D) + lane);
-      cv[0] = v4.x; cv[1 % PER] = v4.y; cv[2 % PER] = v4.z; cv[3 % PER] = v4.w;
-    } else {
-      const float2 v2 = __ldg(reinterpret_cast<const float2*>(crow + (size_t)t * D) + lane);
-      cv[0] = v2.x; cv[1 % PER] = v2.y;
-    }
-#pragma unroll
-    for (int hh = 0; hh < grp; ++hh) {
-      float s = 0.f;
-#pragma unroll
-      for (int a = 0; a < PER; ++a) s = fmaf(qreg[hh][a], cv[a], s);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-      if (lane == 0) sc[(size_t)hh * nb + t] = s;
-    }
-  }
   __syncthreads();
   const int ncand = p.force_last ? nb - 1 : nb;
   for (int hh = 0; hh < grp; ++hh) {

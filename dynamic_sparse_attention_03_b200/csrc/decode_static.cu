@@ -56,6 +56,8 @@ int launch(const DecodeParams& p, int B, int Hkv, int nchmax, size_t sel_smem, c
       cudaFuncSetAttribute(decode_select_kernel<D, G, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)sel_smem) != cudaSuccess)
     return DSA_ERR_CUDA;
+  decode_score_kernel<D, G><<<dim3(B * Hkv, (p.nb + 63) / 64), 256, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   decode_select_kernel<D, G, 256><<<B * Hkv, 256, sel_smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (cudaFuncSetAttribute(decode_attn_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -87,11 +89,11 @@ extern "C" int sparse_decode_attn_static(const void* q, const void* k_cache, con
   const int ncand = force_last ? nb - 1 : nb;
   const int count = (keep < ncand ? keep : ncand) + force_last;
   if (sel_idx && kcap < count) return DSA_ERR_CAPACITY;
-  const size_t sel_smem = (size_t)grp * d * 4 + (size_t)grp * nb * 4 + (size_t)nb * 4 + nb;
+  const size_t sel_smem = (size_t)grp * nb * 4 + (size_t)nb * 4 + nb;
   if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
   const int nchmax = (nb + kDecChunk - 1) / kDecChunk;
   // Scratch layout (same as the workspace of sparse_decode_attn): status word,
-  // union lists and masks, union counts, chunk partials.
+  // union lists and masks, union counts, chunk partials, block scores.
   size_t off = 0;
   const size_t o_status = off; off = up256(off + 256);
   const size_t o_uidx = off;   off = up256(off + (size_t)B * Hkv * nb * 4);
@@ -99,6 +101,7 @@ extern "C" int sparse_decode_attn_static(const void* q, const void* k_cache, con
   const size_t o_ucnt = off;   off = up256(off + (size_t)B * Hkv * 4);
   const size_t o_ml = off;     off = up256(off + (size_t)B * Hq * nchmax * 2 * 4);
   const size_t o_acc = off;    off = up256(off + (size_t)B * Hq * nchmax * d * 4);
+  const size_t o_sc = off;     off = up256(off + (size_t)B * Hq * nb * 4);
   if (off > kStaticScratchBytes) return DSA_ERR_CAPACITY;
   uint8_t* base = static_cast<uint8_t*>(scratch_on_current_device());
   if (!base) return DSA_ERR_CUDA;
@@ -112,6 +115,7 @@ extern "C" int sparse_decode_attn_static(const void* q, const void* k_cache, con
   p.ucnt = reinterpret_cast<int32_t*>(base + o_ucnt);
   p.part_ml = reinterpret_cast<float*>(base + o_ml);
   p.part_acc = reinterpret_cast<float*>(base + o_acc);
+  p.scores = reinterpret_cast<float*>(base + o_sc);
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.kc = static_cast<const __nv_bfloat16*>(k_cache);
   p.vc = static_cast<const __nv_bfloat16*>(v_cache);
