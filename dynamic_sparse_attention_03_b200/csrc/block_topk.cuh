@@ -12,9 +12,10 @@
 // lane, 64 columns each).  Rather than storing the scores, the kernel
 // recomputes them in passes:
 //
-//   pass 0 (approximate, Q̄hi·K̄hi only): min, max, mean and spread of a 1/4
-//           sample of the row (the first 32 columns of every chunk), which
-//           place a 256-bin value window over the row;
+//   pass 0 (approximate, Q̄hi·K̄hi only): min, max, mean and spread of a
+//           sample of the row (the first 32 columns of every 4th chunk), which
+//           place a 256-bin value window over the row; rows of at most four
+//           chunks are read whole and the window is their range;
 //   pass 1 (approximate): a 256-bin histogram of the row in that window gives
 //           the bin holding the row's e-th largest score;
 //   pass 2 (exact, 3xTF32): scores above that bin (widened by a quarter bin on
@@ -100,7 +101,7 @@ __device__ __forceinline__ bool topk_hist_mode(int m) { return m == kSelAHist ||
 
 struct TopkRow {
   int i, L, e, mode;
-  float inv, nlo;              // value bin = floor(s * inv + nlo), clamped to [0, 255]
+  float inv, nlo;              // value bin = round(255 * sat(s * inv + nlo)), see topk_bin
   float wlo, whi;              // window of the exact pass
   float mn, mx, sum, sq, cnt;  // approximate statistics of the sample
   int b0;                      // boundary value bin (fallback)
@@ -123,14 +124,19 @@ struct TopkPub {
   int cnt2[128];   // second thread: nd | nc << 16
 };
 
-// Value bin in [0, 255]: s * inv + nlo clamped to [-1, 256] and rounded to
-// the nearest integer by adding 1.5 * 2^23 (no float-to-int conversion
-// instruction).  Every step is monotone in s, so the bin order is the score
-// order; all passes that compare bins use this same function.
+// Value bin in [0, 255]: y = s * inv + nlo saturated to [0, 1] (a NaN gives
+// 0), then b = 255 y rounded to the nearest integer by adding 1.5 * 2^23 in
+// the same multiply-add (no float-to-int conversion).  topk_bin_bits returns
+// the float's bits, 0x4B400000 + b, whose low 8 bits are b.  Every step is
+// monotone in s, so the bin order is the score order; all passes that compare
+// bins use this same function.  A window [lo, hi] has inv = 1 / (hi - lo) and
+// nlo = -lo * inv; bin b then holds the scores near lo + b (hi - lo) / 255.
+__device__ __forceinline__ uint32_t topk_bin_bits(float s, float inv, float nlo) {
+  const float y = __saturatef(fmaf(s, inv, nlo));
+  return __float_as_uint(fmaf(y, 255.f, 12582912.f));
+}
 __device__ __forceinline__ int topk_bin(float s, float inv, float nlo) {
-  const float x = fminf(fmaxf(fmaf(s, inv, nlo), -1.f), 256.f);
-  const int b = __float_as_int(x + 12582912.f) - 0x4B400000;
-  return min(max(b, 0), 255);
+  return (int)(topk_bin_bits(s, inv, nlo) - 0x4B400000u);
 }
 
 // Private per-row words in shared memory: word w of row r at [w][r] (row r's
@@ -148,12 +154,17 @@ __device__ __forceinline__ void hist_clear(const RowWords& W) {
   for (int w = 0; w < 128; ++w) W[w] = 0u;
 }
 
-// Adds 1 to bin b when `on` (else adds 0): a shared-memory atomic whose
-// result is unused, so consecutive adds to one word do not wait on each
-// other's load and store; both threads of a row add into the same words.
-__device__ __forceinline__ void hist_add_if(const RowWords& W, int b, bool on) {
-  const uint32_t inc = on ? (1u << ((b & 1) << 4)) : 0u;
-  atomicAdd(&W[b >> 1], inc);   // result unused: a shared-memory reduction
+// 16-bit bin counts, two per word: bins b and b + 128 share word b & 127
+// (low and high half).  Adds 1 to bin (b & 255) when `on` (else adds 0): a
+// shared-memory atomic whose result is unused, so consecutive adds to one
+// word do not wait on each other's load and store; both threads of a row add
+// into the same words.  b may carry bits above the low 8 (topk_bin_bits).
+__device__ __forceinline__ void hist_add_if(const RowWords& W, uint32_t b, bool on) {
+  const uint32_t inc = on ? ((b & 128u) ? 65536u : 1u) : 0u;
+  atomicAdd(&W[b & 127u], inc);   // result unused: a shared-memory reduction
+}
+__device__ __forceinline__ void hist_add(const RowWords& W, uint32_t b) {
+  atomicAdd(&W[b & 127u], (b & 128u) ? 65536u : 1u);
 }
 
 // Upper-tail quantile of the standard normal: z with P(Z > z) = q, from the
@@ -175,21 +186,24 @@ __device__ __forceinline__ void hist_find(const RowWords& W, int t, int& bin, in
   bin = 0;
   cnt = 0;
 #pragma unroll 4
-  for (int w = 127; w >= 0; --w) {
-    const uint32_t word = W[w];
-    const int chi = (int)(word >> 16), clo = (int)(word & 0xFFFFu);
-    if (above + chi >= t) {
-      bin = 2 * w + 1;
-      cnt = chi;
+  for (int w = 127; w >= 0; --w) {   // bins 255 .. 128: high halves
+    const int c = (int)(W[w] >> 16);
+    if (above + c >= t) {
+      bin = 128 + w;
+      cnt = c;
       return;
     }
-    above += chi;
-    if (above + clo >= t) {
-      bin = 2 * w;
-      cnt = clo;
+    above += c;
+  }
+#pragma unroll 4
+  for (int w = 127; w >= 0; --w) {   // bins 127 .. 0: low halves
+    const int c = (int)(W[w] & 0xFFFFu);
+    if (above + c >= t) {
+      bin = w;
+      cnt = c;
       return;
     }
-    above += clo;
+    above += c;
   }
 }
 
@@ -243,16 +257,34 @@ __device__ __forceinline__ void topk_resolve(const RowWords& W, int ncA, int ncB
   }
 }
 
-// Buffers the candidates `in` of a group at slots base + nc, ...: key and id.
+// v[t] for a run-time t: a five-level select tree on the bits of t (an
+// indexed register array would live in local memory).
+__device__ __forceinline__ uint32_t select32(const uint32_t (&v)[32], int t) {
+  uint32_t a[16], b[8], c[4], d[2];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) a[k] = (t & 1) ? v[2 * k + 1] : v[2 * k];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) b[k] = (t & 2) ? a[2 * k + 1] : a[2 * k];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) c[k] = (t & 4) ? b[2 * k + 1] : b[2 * k];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) d[k] = (t & 8) ? c[2 * k + 1] : c[2 * k];
+  return (t & 16) ? d[1] : d[0];
+}
+
+// Buffers the candidates `in` of a group at slots base + nc, ...: key and id
+// (candidates are few per group: one select per candidate).  Slots past
+// kTopkCap are counted but not stored.
 __device__ __forceinline__ void topk_buffer(const uint32_t (&v)[32], uint32_t in, int base, int nc, int jx,
                                             const RowWords& W) {
-#pragma unroll
-  for (int t = 0; t < 32; ++t) {
-    const int slot = nc + __popc(in & ((1u << t) - 1u));
-    if (((in >> t) & 1u) && slot < kTopkCap) {
-      W[base + slot] = float_key(__uint_as_float(v[t]));
-      W[64 + base + slot] = (uint32_t)(jx + t);
+  while (in) {
+    const int t = __ffs(in) - 1;
+    in &= in - 1u;
+    if (nc < kTopkCap) {
+      W[base + nc] = float_key(__uint_as_float(select32(v, t)));
+      W[64 + base + nc] = (uint32_t)(jx + t);
     }
+    ++nc;
   }
 }
 
@@ -275,10 +307,14 @@ __device__ __forceinline__ void topk_accum32(TopkRow& R, const uint32_t (&v)[32]
     }
     R.cnt += (float)__popc(valid);
   } else if (R.mode == kSelAHist || R.mode == kSelHist) {
+    if (valid == 0xFFFFFFFFu) {
+      // whole group: two multiply-adds, the word and the half, one add each
 #pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      const int b = topk_bin(__uint_as_float(v[t]), R.inv, R.nlo);
-      hist_add_if(W, b, (valid >> t) & 1u);
+      for (int t = 0; t < 32; ++t) hist_add(W, topk_bin_bits(__uint_as_float(v[t]), R.inv, R.nlo));
+    } else {
+#pragma unroll
+      for (int t = 0; t < 32; ++t)
+        hist_add_if(W, topk_bin_bits(__uint_as_float(v[t]), R.inv, R.nlo), (valid >> t) & 1u);
     }
   } else if (R.mode == kSelRadix) {
 #pragma unroll
@@ -286,7 +322,7 @@ __device__ __forceinline__ void topk_accum32(TopkRow& R, const uint32_t (&v)[32]
       const float s = __uint_as_float(v[t]);
       const uint32_t k = float_key(s);
       const bool member = ((valid >> t) & 1u) && topk_bin(s, R.inv, R.nlo) == R.b0 && (k & R.mask) == R.prefix;
-      hist_add_if(W, (int)((k >> R.shift) & 255u), member);
+      hist_add_if(W, (k >> R.shift) & 255u, member);
     }
   }
 }
@@ -429,7 +465,8 @@ __device__ __forceinline__ void topk_emit_row(const TopkParams& p, int h, int i,
 // Warps: 0 = TMA producer (Q̄ per tile, then K̄), 1 = MMA issuer, 2..5 =
 // first threads of the 128 rows (own the row's selection state; columns 0..63
 // of each chunk), 6..9 = second threads (columns 64..127).  The statistics
-// pass reads columns 0..31 (first threads); the exact fallback that keeps
+// pass reads columns 0..31 (all 128 in tiles of at most 4 chunks; first
+// threads); the exact fallback that keeps
 // threshold-valued ids in column order reads all 128 columns (first threads).
 // Warp w reads TMEM lane quarter w % 4.
 template <int D>
@@ -666,7 +703,7 @@ __global__ void __launch_bounds__(320, 1)
         const bool keeps = (m == kSelWindow || m == kSelCollect || m == kSelExact);
         // column groups of 32 this thread reads in this pass
         uint32_t need;
-        if (m == kSelStats) need = second ? 0u : 0x1u;
+        if (m == kSelStats) need = second ? 0u : (nch <= 4 ? 0xFu : 0x1u);
         else if (m == kSelExact) need = second ? 0u : 0xFu;
         else if (topk_hist_mode(m) || keeps) need = second ? 0xCu : 0x3u;
         else need = 0u;
@@ -732,7 +769,9 @@ __global__ void __launch_bounds__(320, 1)
           switch (R.mode) {
             case kSelStats: {
               float lo = R.mn, hi = R.mx;
-              if (R.cnt > 0.f && R.sum == R.sum && R.mn <= R.mx) {
+              // rows of at most 4 chunks were read whole: their window is the
+              // row's range (a few scores per bin); longer rows were sampled
+              if (nch > 4 && R.cnt > 0.f && R.sum == R.sum && R.mn <= R.mx) {
                 // the sample's mean and spread place the window: from one
                 // spread below the estimated e-th largest score (a normal
                 // model of the row) to six spreads above the mean
@@ -746,7 +785,7 @@ __global__ void __launch_bounds__(320, 1)
                   hi = R.mx;
                 }
               }
-              float inv = (hi > lo) ? 256.f / (hi - lo) : 0.f;
+              float inv = (hi > lo) ? 1.f / (hi - lo) : 0.f;
               if (!(inv <= 3.0e38f)) inv = 0.f;
               R.inv = inv;
               R.nlo = (inv > 0.f) ? -lo * inv : 0.f;
@@ -758,9 +797,11 @@ __global__ void __launch_bounds__(320, 1)
               hist_find(W, R.e, bin, above, cnt);
               const float kInf = __int_as_float(0x7f800000);
               if (R.inv > 0.f) {
-                const float lo = -R.nlo / R.inv;
-                R.wlo = (bin == 0) ? -kInf : lo + ((float)bin - 0.75f) / R.inv;
-                R.whi = (bin == 255) ? kInf : lo + ((float)bin + 0.75f) / R.inv;
+                // bin b holds y in [(b - 1/2) / 255, (b + 1/2) / 255): the exact
+                // window reaches a quarter bin further on each side
+                const float lo = -R.nlo / R.inv, w = 1.f / (255.f * R.inv);
+                R.wlo = (bin == 0) ? -kInf : lo + ((float)bin - 0.75f) * w;
+                R.whi = (bin == 255) ? kInf : lo + ((float)bin + 0.75f) * w;
               } else {
                 R.wlo = -kInf;
                 R.whi = kInf;
