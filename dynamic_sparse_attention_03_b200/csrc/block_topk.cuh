@@ -155,16 +155,20 @@ __device__ __forceinline__ void hist_clear(const RowWords& W) {
 }
 
 // 16-bit bin counts, two per word: bins b and b + 128 share word b & 127
-// (low and high half).  Adds 1 to bin (b & 255) when `on` (else adds 0): a
-// shared-memory atomic whose result is unused, so consecutive adds to one
-// word do not wait on each other's load and store; both threads of a row add
-// into the same words.  b may carry bits above the low 8 (topk_bin_bits).
-__device__ __forceinline__ void hist_add_if(const RowWords& W, uint32_t b, bool on) {
-  const uint32_t inc = on ? ((b & 128u) ? 65536u : 1u) : 0u;
-  atomicAdd(&W[b & 127u], inc);   // result unused: a shared-memory reduction
-}
+// (low and high half).  Adds 1 to bin (b & 255), when `on` for hist_add_if:
+// a shared-memory reduction (red, no result), so consecutive adds to one word
+// do not wait on each other; both threads of a row add into the same words.
+// b may carry bits above the low 8 (topk_bin_bits).  The words are read only
+// after a barrier, which orders these adds before the reads.
 __device__ __forceinline__ void hist_add(const RowWords& W, uint32_t b) {
-  atomicAdd(&W[b & 127u], (b & 128u) ? 65536u : 1u);
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(W.addr((int)(b & 127u))), "r"((b & 128u) ? 65536u : 1u));
+}
+__device__ __forceinline__ void hist_add_if(const RowWords& W, uint32_t b, bool on) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %2, 0;\n\t"
+      "@p red.shared.add.u32 [%0], %1;\n\t}" ::"r"(W.addr((int)(b & 127u))),
+      "r"((b & 128u) ? 65536u : 1u), "r"((uint32_t)on));
 }
 
 // Upper-tail quantile of the standard normal: z with P(Z > z) = q, from the
@@ -181,29 +185,36 @@ __device__ __forceinline__ float normal_upper_quantile(float q) {
 
 // Bin holding the t-th largest element (1 <= t <= total), scanning 16-bit
 // counts from the top: returns the bin, the count strictly above it and its own.
+// Words are read 8 at a time (independent loads) and the batch's total is
+// tested before its bins.
 __device__ __forceinline__ void hist_find(const RowWords& W, int t, int& bin, int& above, int& cnt) {
   above = 0;
   bin = 0;
   cnt = 0;
-#pragma unroll 4
-  for (int w = 127; w >= 0; --w) {   // bins 255 .. 128: high halves
-    const int c = (int)(W[w] >> 16);
-    if (above + c >= t) {
-      bin = 128 + w;
-      cnt = c;
-      return;
+#pragma unroll 1
+  for (int half = 1; half >= 0; --half) {   // bins 255 .. 128 (high halves), then 127 .. 0
+    const int sh = 16 * half;
+#pragma unroll 1
+    for (int w0 = 127; w0 >= 0; w0 -= 8) {
+      int c[8], tot = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        c[k] = (int)((W[w0 - k] >> sh) & 0xFFFFu);
+        tot += c[k];
+      }
+      if (above + tot >= t) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (above + c[k] >= t) {
+            bin = 128 * half + w0 - k;
+            cnt = c[k];
+            return;
+          }
+          above += c[k];
+        }
+      }
+      above += tot;
     }
-    above += c;
-  }
-#pragma unroll 4
-  for (int w = 127; w >= 0; --w) {   // bins 127 .. 0: low halves
-    const int c = (int)(W[w] & 0xFFFFu);
-    if (above + c >= t) {
-      bin = w;
-      cnt = c;
-      return;
-    }
-    above += c;
   }
 }
 
@@ -251,8 +262,7 @@ __device__ __forceinline__ void topk_resolve(const RowWords& W, int ncA, int ncB
   for (int x = 0; x < nc; ++x) {
     if (all || W[slot(x)] > T || ((taken >> x) & 1ull)) {
       const int j = (int)W[64 + slot(x)];
-      uint32_t* wd = mrow + (j >> 7) * 4 + ((j & 127) >> 5);
-      *wd |= 1u << (j & 31);
+      atomicOr(mrow + (j >> 7) * 4 + ((j & 127) >> 5), 1u << (j & 31));   // no result: a reduction
     }
   }
 }
