@@ -82,15 +82,15 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t rows, int d) {
   return r == CUDA_SUCCESS;
 }
 
-// 2D fp32 view [rows][d] with a 32-float (128-byte) x box_rows box and 128-byte swizzle.
-bool make_tmap_f32(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
+// 2D fp16 view [rows][d] with a 64-element (128-byte) x box_rows box and 128-byte swizzle.
+bool make_tmap_f16(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 4};
-  cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -247,18 +247,22 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   }
   WsCarve c(ws);
   uint32_t* status = static_cast<uint32_t*>(c.take(kStatusBytes));
-  // TF32 hi/lo halves of the pooled means, the operands of the tensor-core scores
-  float* q_hi = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hq * nQB * d * 4));
-  float* q_lo = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hq * nQB * d * 4));
-  float* k_hi = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hkv * nQB * d * 4));
-  float* k_lo = pool_only ? nullptr : static_cast<float*>(c.take((size_t)Hkv * nQB * d * 4));
+  // FP16 hi/lo halves of the scaled pooled means, the operands of the
+  // tensor-core scores (scales: per query block for Q, per KV head for K)
+  __half* q_hi = pool_only ? nullptr : static_cast<__half*>(c.take((size_t)Hq * nQB * d * 2));
+  __half* q_lo = pool_only ? nullptr : static_cast<__half*>(c.take((size_t)Hq * nQB * d * 2));
+  __half* k_hi = pool_only ? nullptr : static_cast<__half*>(c.take((size_t)Hkv * nQB * d * 2));
+  __half* k_lo = pool_only ? nullptr : static_cast<__half*>(c.take((size_t)Hkv * nQB * d * 2));
   float* kbar = pooled_k;
+  if (!pool_only && !kbar) kbar = static_cast<float*>(c.take((size_t)Hkv * nQB * d * 4));
+  // per KV head max |K̄| (float bits) and the top-k tile counter, zeroed together
+  unsigned* kmax = pool_only ? nullptr : static_cast<unsigned*>(c.take((size_t)(Hkv + 1) * 4));
   // kept-column bit masks written by the fused score/top-k kernel and read by
   // the list kernel: 16 bytes per (head, query block, key chunk of its tile)
   const int nrt = (nQB + 127) / 128;
   uint32_t* masks = pool_only ? nullptr
                               : static_cast<uint32_t*>(c.take((size_t)Hq * topk_mask_words_per_head(nrt) * 4));
-  int* next_tile = pool_only ? nullptr : static_cast<int*>(c.take(sizeof(int)));
+  int* next_tile = pool_only ? nullptr : reinterpret_cast<int*>(kmax + Hkv);
   if (!ws) {
     *ws_bytes = c.off;
     return DSA_OK;
@@ -267,15 +271,18 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
   const int64_t nkb = (int64_t)Hkv * nQB, nqb = (int64_t)Hq * nQB;
-  if (d == 128) pool_blocks_kernel<128><<<(unsigned)nkb, 256, 0, st>>>(kb, kbar, nkb, k_hi, k_lo);
-  else pool_blocks_kernel<64><<<(unsigned)nkb, 256, 0, st>>>(kb, kbar, nkb, k_hi, k_lo);
+  if (!pool_only && cudaMemsetAsync(kmax, 0, (size_t)(Hkv + 1) * 4, st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (d == 128)
+    pool_blocks_kernel<128><<<(unsigned)nkb, 256, 0, st>>>(kb, kbar, nkb, kmax, nQB, nullptr, nullptr, nullptr, 0,
+                                                           nullptr, nullptr, nullptr);
+  else
+    pool_blocks_kernel<64><<<(unsigned)nkb, 256, 0, st>>>(kb, kbar, nkb, kmax, nQB, nullptr, nullptr, nullptr, 0,
+                                                          nullptr, nullptr, nullptr);
   if (int rc = launch_check()) return rc;
   if (pool_only) return DSA_OK;
   const auto* qp = static_cast<const __nv_bfloat16*>(q);
-  CUtensorMap tqh, tql, tkh, tkl;
-  if (!make_tmap_f32(&tqh, q_hi, nqb, d, 128) || !make_tmap_f32(&tql, q_lo, nqb, d, 128) ||
-      !make_tmap_f32(&tkh, k_hi, nkb, d, 128) || !make_tmap_f32(&tkl, k_lo, nkb, d, 128))
-    return DSA_ERR_CUDA;
+  CUtensorMap tkh, tkl;
+  if (!make_tmap_f16(&tkh, k_hi, nkb, d, 128) || !make_tmap_f16(&tkl, k_lo, nkb, d, 128)) return DSA_ERR_CUDA;
   TopkParams tp{};
   tp.block_idx = block_idx;
   tp.block_cnt = block_cnt;
@@ -288,6 +295,8 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   tp.nrt = nrt;
   tp.masks = masks;
   tp.ppm = ppm;
+  tp.qhi = q_hi;
+  tp.qlo = q_lo;
   int dev = 0, nsm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
@@ -296,8 +305,15 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   if ((rc = (d == 128) ? set_smem(block_topk_kernel<128>, TopkLayout<128>::kSmemAlloc)
                        : set_smem(block_topk_kernel<64>, TopkLayout<64>::kSmemAlloc)))
     return rc;
-  if (d == 128) pool_blocks_kernel<128><<<(unsigned)nqb, 256, 0, st>>>(qp, nullptr, nqb, q_hi, q_lo);
-  else pool_blocks_kernel<64><<<(unsigned)nqb, 256, 0, st>>>(qp, nullptr, nqb, q_hi, q_lo);
+  // Q pooling (split with each query block's own scale), then 8 pooled-key
+  // rows per extra CTA split with their KV head's scale
+  const unsigned qgrid = (unsigned)(nqb + (nkb + 7) / 8);
+  if (d == 128)
+    pool_blocks_kernel<128><<<qgrid, 256, 0, st>>>(qp, nullptr, nqb, nullptr, nQB, q_hi, q_lo, kbar, nkb, kmax,
+                                                   k_hi, k_lo);
+  else
+    pool_blocks_kernel<64><<<qgrid, 256, 0, st>>>(qp, nullptr, nqb, nullptr, nQB, q_hi, q_lo, kbar, nkb, kmax,
+                                                  k_hi, k_lo);
   if ((rc = launch_check())) return rc;
   // pooled scores and the per-row top-k in one kernel (the scores stay on chip)
   tp.h0 = 0;
@@ -305,9 +321,8 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   tp.ntiles = nrt * Hq;
   tp.next_tile = next_tile;
   const unsigned grid = (unsigned)std::min(std::min(nsm, kTopkMaxGrid), tp.ntiles);
-  if (cudaMemsetAsync(next_tile, 0, sizeof(int), st) != cudaSuccess) return DSA_ERR_CUDA;
-  if (d == 128) block_topk_kernel<128><<<grid, 320, TopkLayout<128>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, tp);
-  else block_topk_kernel<64><<<grid, 320, TopkLayout<64>::kSmemAlloc, st>>>(tqh, tql, tkh, tkl, tp);
+  if (d == 128) block_topk_kernel<128><<<grid, 320, TopkLayout<128>::kSmemAlloc, st>>>(tkh, tkl, tp);
+  else block_topk_kernel<64><<<grid, 320, TopkLayout<64>::kSmemAlloc, st>>>(tkh, tkl, tp);
   if ((rc = launch_check())) return rc;
   const int64_t nrows = (int64_t)Hq * nQB;
   // rows of the last row tile have 4 nrt mask words: 32-word batches

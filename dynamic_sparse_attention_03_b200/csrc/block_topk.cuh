@@ -5,8 +5,9 @@
 // ties to the lower block).
 //
 // A persistent grid walks tiles of (q-head, 128 query blocks), heaviest first.
-// A tile's Q̄ (TF32 hi and lo halves) sits in tensor memory as the A operand;
-// the KV head's K̄ streams through a TMA ring in chunks of 128 key blocks;
+// A tile's Q̄ (FP16 hi and lo halves of the scaled means, see
+// pool_blocks_kernel) sits in tensor memory as the A operand; the KV head's K̄
+// (FP16 hi and lo) streams through a TMA ring in chunks of 128 key blocks;
 // S = Q̄·K̄ᵀ for a chunk is computed with tcgen05 into one of two TMEM buffers,
 // and each query block's row of the chunk is read by two threads (one TMEM
 // lane, 64 columns each).  Rather than storing the scores, the kernel
@@ -18,7 +19,7 @@
 //           chunks are read whole and the window is their range;
 //   pass 1 (approximate): a 256-bin histogram of the row in that window gives
 //           the bin holding the row's e-th largest score;
-//   pass 2 (exact, 3xTF32): scores above that bin (widened by a quarter bin on
+//   pass 2 (exact: Q̄hi·K̄hi + Q̄hi·K̄lo + Q̄lo·K̄hi): scores above that bin (widened by a quarter bin on
 //           each side) are kept at once, as bits of a per-chunk mask in
 //           scratch memory; scores inside it are buffered as (key, id)
 //           candidates.  If the kept count and the candidates bracket e, the
@@ -38,6 +39,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "index_kernels.cuh"
@@ -47,7 +49,7 @@ namespace dsa {
 
 template <int D>
 struct TopkLayout {
-  static constexpr int kStages = 8;                 // ring of stages, each 128 rows x 32 fp32
+  static constexpr int kStages = 8;                 // ring of stages, each 128 key blocks x 64 fp16
   static constexpr int kTile = 128 * 128;
   static constexpr int kRow = kStages * kTile;      // per-row private words: [128 words][128 rows] u32
   static constexpr int kRowBytes = 128 * 128 * 4;
@@ -57,9 +59,8 @@ struct TopkLayout {
   static constexpr int kCtl = kBar + 256;
   static constexpr int kBytes = kCtl + 64;
   static constexpr int kSmemAlloc = kBytes + 1024;
-  static constexpr int NDC = D / 32;                // d chunks of 32 floats
-  static_assert(NDC * kTile <= kRowBytes, "Q hi tile staged in the per-row region");
-  static_assert(NDC <= kStages / 2, "Q lo tile staged in the first ring stages");
+  static constexpr int NDC = D / 64;                // d chunks of 64 fp16 (one 128-byte swizzled row)
+  static_assert(NDC >= 1 && NDC <= 2, "D is 64 or 128");
 };
 
 constexpr int kTopkCap = 32;         // buffered boundary candidates per row thread
@@ -74,14 +75,16 @@ struct TopkParams {
   int nQB, Hq, grp, kcap, k_fixed, nrt, ntiles;
   int h0, nh;          // q-heads h0 .. h0 + nh - 1 are this launch's (ntiles = nrt * nh)
   int64_t ppm;
+  const __half* qhi;   // [Hq * nQB][D] FP16 halves of the scaled query-block means
+  const __half* qlo;
 };
 
-__device__ __forceinline__ void umma_tf32_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
-                                             uint32_t accumulate) {
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
       "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -185,36 +188,54 @@ __device__ __forceinline__ float normal_upper_quantile(float q) {
 
 // Bin holding the t-th largest element (1 <= t <= total), scanning 16-bit
 // counts from the top: returns the bin, the count strictly above it and its own.
-// Words are read 8 at a time (independent loads) and the batch's total is
-// tested before its bins.
+// Two levels, without data-dependent branches until the end: the totals of
+// the 32 batches of 8 bins (each word loaded once, both halves summed), then
+// the batch holding the t-th element, then its 8 bins.
 __device__ __forceinline__ void hist_find(const RowWords& W, int t, int& bin, int& above, int& cnt) {
-  above = 0;
+  int tot[32];   // tot[j]: bins 8j .. 8j+7 (j >= 16: high halves of words 8(j-16) ..)
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    int lo = 0, hi = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t x = W[8 * j + k];
+      lo += (int)(x & 0xFFFFu);
+      hi += (int)(x >> 16);
+    }
+    tot[j] = lo;
+    tot[16 + j] = hi;
+  }
+  int acc = 0, jb = 0, ab = 0;
+  bool found = false;
+#pragma unroll
+  for (int j = 31; j >= 0; --j) {
+    const bool here = !found && acc + tot[j] >= t;
+    jb = here ? j : jb;
+    ab = here ? acc : ab;
+    found = found || here;
+    acc += tot[j];
+  }
+  above = ab;
   bin = 0;
   cnt = 0;
-#pragma unroll 1
-  for (int half = 1; half >= 0; --half) {   // bins 255 .. 128 (high halves), then 127 .. 0
-    const int sh = 16 * half;
-#pragma unroll 1
-    for (int w0 = 127; w0 >= 0; w0 -= 8) {
-      int c[8], tot = 0;
+  if (!found) {   // fewer than t elements in all: bin 0, everything above it
+    above = acc;
+    return;
+  }
+  const int sh = jb >= 16 ? 16 : 0, w0 = 8 * (jb & 15);
+  int c[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        c[k] = (int)((W[w0 - k] >> sh) & 0xFFFFu);
-        tot += c[k];
-      }
-      if (above + tot >= t) {
+  for (int k = 0; k < 8; ++k) c[k] = (int)((W[w0 + k] >> sh) & 0xFFFFu);
+  bool got = false;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (above + c[k] >= t) {
-            bin = 128 * half + w0 - k;
-            cnt = c[k];
-            return;
-          }
-          above += c[k];
-        }
-      }
-      above += tot;
+  for (int k = 7; k >= 0; --k) {
+    const bool here = !got && above + c[k] >= t;
+    if (here) {
+      bin = 8 * jb + k;
+      cnt = c[k];
     }
+    if (!got && !here) above += c[k];
+    got = got || here;
   }
 }
 
@@ -472,7 +493,7 @@ __device__ __forceinline__ void topk_emit_row(const TopkParams& p, int h, int i,
   if (lane == 0) p.block_cnt[(size_t)h * p.nQB + i] = cnt;
 }
 
-// Warps: 0 = TMA producer (Q̄ per tile, then K̄), 1 = MMA issuer, 2..5 =
+// Warps: 0 = TMA producer (K̄), 1 = MMA issuer, 2..5 =
 // first threads of the 128 rows (own the row's selection state; columns 0..63
 // of each chunk), 6..9 = second threads (columns 64..127).  The statistics
 // pass reads columns 0..31 (all 128 in tiles of at most 4 chunks; first
@@ -481,8 +502,7 @@ __device__ __forceinline__ void topk_emit_row(const TopkParams& p, int h, int i,
 // Warp w reads TMEM lane quarter w % 4.
 template <int D>
 __global__ void __launch_bounds__(320, 1)
-    block_topk_kernel(const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmQl,
-                      const __grid_constant__ CUtensorMap tmKh, const __grid_constant__ CUtensorMap tmKl,
+    block_topk_kernel(const __grid_constant__ CUtensorMap tmKh, const __grid_constant__ CUtensorMap tmKl,
                       const TopkParams p) {
   using Lay = TopkLayout<D>;
   extern __shared__ uint8_t tk_smem_raw[];
@@ -495,7 +515,7 @@ __global__ void __launch_bounds__(320, 1)
   auto bempty = [&](int s) { return bar0 + 8u * (8 + s); };
   auto sfull = [&](int b) { return bar0 + 8u * (16 + b); };
   auto sempty = [&](int b) { return bar0 + 8u * (18 + b); };
-  const uint32_t qfull = bar0 + 160u, qready = bar0 + 168u, done = bar0 + 176u;
+  const uint32_t qready = bar0 + 168u, done = bar0 + 176u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kCtl);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kCtl + 4);
   volatile int* tile_slot = reinterpret_cast<volatile int*>(smem + Lay::kCtl + 8);
@@ -507,7 +527,6 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(sfull(1), 1);
     mbar_init(sempty(0), 8);
     mbar_init(sempty(1), 8);
-    mbar_init(qfull, 1);
     mbar_init(qready, 8);
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -524,8 +543,8 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
   const AbortState ab{abort_flag, p.status};
   const bool issuer = elect_one();   // the MMA warp's issuing lane (also its committer)
-  constexpr uint32_t kColQh = 256, kColQl = 256 + D;
-  constexpr int GA = Lay::NDC;       // stages per group: approximate passes (a chunk's hi)
+  constexpr uint32_t kColQh = 256, kColQl = 256 + D / 2;   // fp16 pairs per TMEM column
+  constexpr int GA = 2;              // stages per group: approximate passes (a chunk's hi, NDC stages used)
   constexpr int GE = 2;              // exact passes (one d chunk's hi and lo)
 
   // ring bookkeeping (producer: next empty-wait parity and issued-but-unreleased
@@ -553,17 +572,6 @@ __global__ void __launch_bounds__(320, 1)
     const int rt = p.nrt - 1 - tile / p.nh;
     const int h = p.h0 + tile % p.nh, g = h / p.grp;
     const int nch = rt + 1;   // key chunks of 128 blocks on or before the tile's diagonal
-    if (warp == 0) {
-      // the tile's Q̄: hi into the per-row region, lo into the first ring stages
-      if (claim(0, Lay::NDC) && lane == 0) {
-        mbar_arrive_expect_tx(qfull, (uint32_t)(2 * Lay::NDC * Lay::kTile));
-        for (int dc = 0; dc < Lay::NDC; ++dc) {
-          tma_load_2d(sb + Lay::kRow + dc * Lay::kTile, &tmQh, dc * 32, h * p.nQB + rt * 128, qfull);
-          tma_load_2d(sb + dc * Lay::kTile, &tmQl, dc * 32, h * p.nQB + rt * 128, qfull);
-        }
-      }
-      __syncwarp();
-    }
 
     // -------------------------------------------------------------- row state
     const bool is_row = warp >= 2;
@@ -583,18 +591,20 @@ __global__ void __launch_bounds__(320, 1)
     R.eq = 0;
     const bool pending0 = valid && !(R.L == 0 || R.e == 0 || R.e >= R.L);
     if (is_row) {
-      // Q̄ of this row from the staged tiles (128-byte swizzle) into TMEM: the
-      // first thread moves the hi half, the second the lo half
-      if (mbar_wait_warp(qfull, (uint32_t)(tcount & 1), ab)) {
-        const uint8_t* src = smem + (second ? 0 : Lay::kRow);
+      // this row's Q̄ from global memory into TMEM (fp16 pairs): the first
+      // thread moves the hi half, the second the lo half; rows past the last
+      // query block get zeros.  The previous tile's MMAs, which read these
+      // columns, completed before its last S buffer was handed over.
+      {
+        const uint4* src = reinterpret_cast<const uint4*>((second ? p.qlo : p.qhi) +
+                                                          (size_t)(h * p.nQB + (valid ? i : 0)) * D);
         const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16) + (second ? kColQl : kColQh);
 #pragma unroll 1
         for (int dc = 0; dc < Lay::NDC; ++dc) {
           uint32_t v[32];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const uint4 q4 =
-                *reinterpret_cast<const uint4*>(src + dc * Lay::kTile + r * 128 + ((k ^ (r & 7)) << 4));
+            const uint4 q4 = valid ? __ldcg(src + dc * 8 + k) : make_uint4(0u, 0u, 0u, 0u);
             v[4 * k] = q4.x;
             v[4 * k + 1] = q4.y;
             v[4 * k + 2] = q4.z;
@@ -627,14 +637,13 @@ __global__ void __launch_bounds__(320, 1)
       if (warp == 0) {
         // ---------------------------------------------------------- K̄ producer
         bool ok = true;
-        if (pass == 0) ok = mbar_wait_warp(qready, (uint32_t)(tcount & 1), ab);   // Q̄ lo left the ring
         for (int c = 0; c < nch && ok && !*abort_flag; c += cstep) {
           if (approx) {
             if (!(ok = claim(spos, GA))) break;
             if (lane == 0) {
-              mbar_arrive_expect_tx(bfull(spos), (uint32_t)(GA * Lay::kTile));
-              for (int dc = 0; dc < GA; ++dc)
-                tma_load_2d(sb + (spos + dc) * Lay::kTile, &tmKh, dc * 32, g * p.nQB + c * 128, bfull(spos));
+              mbar_arrive_expect_tx(bfull(spos), (uint32_t)(Lay::NDC * Lay::kTile));
+              for (int dc = 0; dc < Lay::NDC; ++dc)
+                tma_load_2d(sb + (spos + dc) * Lay::kTile, &tmKh, dc * 64, g * p.nQB + c * 128, bfull(spos));
             }
             pend |= 1u << spos;
             spos = (spos + GA) & (Lay::kStages - 1);
@@ -643,8 +652,8 @@ __global__ void __launch_bounds__(320, 1)
               if (!(ok = claim(spos, GE))) break;
               if (lane == 0) {
                 mbar_arrive_expect_tx(bfull(spos), (uint32_t)(GE * Lay::kTile));
-                tma_load_2d(sb + spos * Lay::kTile, &tmKh, dc * 32, g * p.nQB + c * 128, bfull(spos));
-                tma_load_2d(sb + (spos + 1) * Lay::kTile, &tmKl, dc * 32, g * p.nQB + c * 128, bfull(spos));
+                tma_load_2d(sb + spos * Lay::kTile, &tmKh, dc * 64, g * p.nQB + c * 128, bfull(spos));
+                tma_load_2d(sb + (spos + 1) * Lay::kTile, &tmKl, dc * 64, g * p.nQB + c * 128, bfull(spos));
               }
               pend |= 1u << spos;
               spos = (spos + GE) & (Lay::kStages - 1);
@@ -656,7 +665,7 @@ __global__ void __launch_bounds__(320, 1)
         // ---------------------------------------------------------- MMA issuer
         // The whole warp walks the issue sequence (warp-uniform operands); the
         // elected lane predicates each instruction.
-        const uint32_t idesc = umma_idesc_tf32(128, 128);
+        const uint32_t idesc = umma_idesc_f16(128, 128);
         bool ok = true;
         if (pass == 0) {
           ok = mbar_wait_warp(qready, (uint32_t)(tcount & 1), ab);
@@ -673,11 +682,11 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after();
             const uint64_t d0 = umma_desc_sw128(sb + spos * Lay::kTile, 16, 1024);
 #pragma unroll
-            for (int dc = 0; dc < GA; ++dc) {
+            for (int dc = 0; dc < Lay::NDC; ++dc) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
+              for (int kk = 0; kk < 4; ++kk) {   // K = 16 fp16 (32 bytes, 8 TMEM columns) per MMA
                 const uint64_t bo = (uint64_t)((dc * Lay::kTile + kk * 32) >> 4);
-                if (issuer) umma_tf32_ts(dS, tmem + kColQh + dc * 32 + kk * 8, d0 + bo, idesc, (dc | kk) ? 1u : 0u);
+                if (issuer) umma_f16_ts(dS, tmem + kColQh + dc * 32 + kk * 8, d0 + bo, idesc, (dc | kk) ? 1u : 0u);
               }
             }
             if (issuer) umma_commit(bempty(spos));
@@ -693,9 +702,9 @@ __global__ void __launch_bounds__(320, 1)
               for (int kk = 0; kk < 4; ++kk) {
                 const uint32_t aH = tmem + kColQh + dc * 32 + kk * 8, aL = tmem + kColQl + dc * 32 + kk * 8;
                 const uint64_t ko = (uint64_t)((kk * 32) >> 4);
-                if (issuer) umma_tf32_ts(dS, aH, dH + ko, idesc, (dc | kk) ? 1u : 0u);
-                if (issuer) umma_tf32_ts(dS, aH, dL + ko, idesc, 1u);
-                if (issuer) umma_tf32_ts(dS, aL, dH + ko, idesc, 1u);
+                if (issuer) umma_f16_ts(dS, aH, dH + ko, idesc, (dc | kk) ? 1u : 0u);
+                if (issuer) umma_f16_ts(dS, aH, dL + ko, idesc, 1u);
+                if (issuer) umma_f16_ts(dS, aL, dH + ko, idesc, 1u);
               }
               if (issuer) umma_commit(bempty(spos));
               spos = (spos + GE) & (Lay::kStages - 1);
@@ -922,7 +931,6 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 0 && lane == 0) {
     for (int t = 0; t < Lay::kStages; ++t)
       if ((pend >> t) & 1u) mbar_wait_cleanup(bempty(t), (eph >> t) & 1u, 200000000ull);
-    if (tcount > 0) mbar_wait_cleanup(qfull, (uint32_t)((tcount - 1) & 1), 200000000ull);
   }
   if (warp == 1) {
     if (issuer) umma_commit(done);
