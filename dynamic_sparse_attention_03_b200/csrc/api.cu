@@ -327,7 +327,7 @@ int sparse_index_estimate(const void* q, const void* k, int Hq, int Hkv, int n, 
   const int64_t nrows = (int64_t)Hq * nQB;
   // rows of the last row tile have 4 nrt mask words: 32-word batches
   const int nbmax = (4 * nrt + 31) / 32;
-  const int64_t list_ctas = std::min<int64_t>((nrows + 7) / 8, (int64_t)nsm * 7);
+  const int64_t list_ctas = std::min<int64_t>((nrows + 7) / 8, (int64_t)nsm * 8);
   if (nbmax <= 2) block_list_kernel<2><<<(unsigned)list_ctas, 256, 0, st>>>(tp);
   else if (nbmax <= 8) block_list_kernel<8><<<(unsigned)list_ctas, 256, 0, st>>>(tp);
   else block_list_kernel<32><<<(unsigned)list_ctas, 256, 0, st>>>(tp);

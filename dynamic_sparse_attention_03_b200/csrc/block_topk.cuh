@@ -434,7 +434,7 @@ __device__ __forceinline__ uint32_t* topk_mask_row(uint32_t* masks, int nrt, int
 
 template <int NB>
 __device__ __forceinline__ void topk_emit_row(const TopkParams& p, int h, int i, const uint32_t (&wv)[NB], int nb,
-                                              int lane, int32_t* stage) {
+                                              int lane) {
   const int L = i > 1 ? i - 1 : 0;
   const int e = extra_budget(i, p.k_fixed, p.ppm);
   int32_t* out = p.block_idx + ((size_t)h * p.nQB + i) * p.kcap;
@@ -452,9 +452,9 @@ __device__ __forceinline__ void topk_emit_row(const TopkParams& p, int h, int i,
     }
     cnt = 2;
   } else {
-    // each batch of 32 mask words (at most 1024 ids) is expanded into the
-    // warp's staging area, then copied out with consecutive lanes on
-    // consecutive ids
+    // each lane holds one mask word of a batch of 32; a warp prefix sum of
+    // the words' counts places each lane's ids, which it writes in order
+    // (no more than e of them: the check below reports a count mismatch)
     int off = 0;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
@@ -467,20 +467,17 @@ __device__ __forceinline__ void topk_emit_row(const TopkParams& p, int h, int i,
         const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
         if (lane >= o) incl += t;
       }
-      int pos = incl - c;
+      int pos = off + incl - c;
       const int w = 32 * b + lane;
       const int jb = (w >> 2) * 128 + (w & 3) * 32;
+      int32_t* dst = out + 1;
       while (word) {
         const int t = __ffs(word) - 1;
         word &= word - 1u;
-        stage[pos++] = jb + t;
+        if (pos < e) dst[pos] = jb + t;
+        ++pos;
       }
-      const int tot = __shfl_sync(0xFFFFFFFFu, incl, 31);
-      __syncwarp();
-      for (int k = lane; k < tot; k += 32)
-        if (off + k < e) out[1 + off + k] = stage[k];
-      __syncwarp();
-      off += tot;
+      off += __shfl_sync(0xFFFFFFFFu, incl, 31);
     }
     if (lane == 0) {
       out[0] = 0;
@@ -599,16 +596,20 @@ __global__ void __launch_bounds__(320, 1)
         const uint4* src = reinterpret_cast<const uint4*>((second ? p.qlo : p.qhi) +
                                                           (size_t)(h * p.nQB + (valid ? i : 0)) * D);
         const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16) + (second ? kColQl : kColQh);
-#pragma unroll 1
+        uint4 q4[Lay::NDC][8];   // every load in flight before the first store
+#pragma unroll
+        for (int dc = 0; dc < Lay::NDC; ++dc)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) q4[dc][k] = valid ? __ldcg(src + dc * 8 + k) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
         for (int dc = 0; dc < Lay::NDC; ++dc) {
           uint32_t v[32];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const uint4 q4 = valid ? __ldcg(src + dc * 8 + k) : make_uint4(0u, 0u, 0u, 0u);
-            v[4 * k] = q4.x;
-            v[4 * k + 1] = q4.y;
-            v[4 * k + 2] = q4.z;
-            v[4 * k + 3] = q4.w;
+            v[4 * k] = q4[dc][k].x;
+            v[4 * k + 1] = q4[dc][k].y;
+            v[4 * k + 2] = q4[dc][k].z;
+            v[4 * k + 3] = q4[dc][k].w;
           }
           tmem_st32(tl + dc * 32, v);
         }
@@ -947,12 +948,11 @@ __global__ void __launch_bounds__(320, 1)
 
 // Writes the block lists from the masks of block_topk_kernel: each warp takes
 // (head, query block) rows in a grid-stride loop, loading the next row's mask
-// words while it writes the current one; 1024 ids of staging per warp.  NB is
+// words while it writes the current one.  NB is
 // the number of 32-word mask batches a row can have (rows of row tile rt have
 // 4 (rt + 1) words), so short rows keep few registers and many warps resident.
 template <int NB>
 __global__ void __launch_bounds__(256) block_list_kernel(const TopkParams p) {
-  __shared__ int32_t stage_all[8][1024];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nrows = (int64_t)p.Hq * p.nQB;
   const int64_t step = (int64_t)gridDim.x * 8;
@@ -975,7 +975,7 @@ __global__ void __launch_bounds__(256) block_list_kernel(const TopkParams p) {
   for (; row < nrows; row += step) {
     const int64_t nrow = row + step;
     if (nrow < nrows) load(nrow, nxt, nbn);
-    topk_emit_row<NB>(p, (int)(row / p.nQB), (int)(row % p.nQB), cur, nbc, lane, stage_all[warp]);
+    topk_emit_row<NB>(p, (int)(row / p.nQB), (int)(row % p.nQB), cur, nbc, lane);
 #pragma unroll
     for (int b = 0; b < NB; ++b) cur[b] = nxt[b];
     nbc = nbn;
