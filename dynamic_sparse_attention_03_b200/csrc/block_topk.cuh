@@ -49,7 +49,7 @@ namespace dsa {
 
 template <int D>
 struct TopkLayout {
-  static constexpr int kStages = 8;                 // ring of stages, each 128 key blocks x 64 fp16
+  static constexpr int kStages = 6;                 // ring of stages, each 128 key blocks x 64 fp16
   static constexpr int kTile = 128 * 128;
   static constexpr int kRow = kStages * kTile;      // per-row private words: [128 words][128 rows] u32
   static constexpr int kRowBytes = 128 * 128 * 4;
@@ -61,6 +61,7 @@ struct TopkLayout {
   static constexpr int kSmemAlloc = kBytes + 1024;
   static constexpr int NDC = D / 64;                // d chunks of 64 fp16 (one 128-byte swizzled row)
   static_assert(NDC >= 1 && NDC <= 2, "D is 64 or 128");
+  static_assert(kStages % 2 == 0, "stages are claimed in pairs");
 };
 
 constexpr int kTopkCap = 32;         // buffered boundary candidates per row thread
@@ -647,7 +648,7 @@ __global__ void __launch_bounds__(320, 1)
                 tma_load_2d(sb + (spos + dc) * Lay::kTile, &tmKh, dc * 64, g * p.nQB + c * 128, bfull(spos));
             }
             pend |= 1u << spos;
-            spos = (spos + GA) & (Lay::kStages - 1);
+            spos = (spos + GA) % Lay::kStages;
           } else {
             for (int dc = 0; dc < Lay::NDC && ok; ++dc) {
               if (!(ok = claim(spos, GE))) break;
@@ -657,7 +658,7 @@ __global__ void __launch_bounds__(320, 1)
                 tma_load_2d(sb + (spos + 1) * Lay::kTile, &tmKl, dc * 64, g * p.nQB + c * 128, bfull(spos));
               }
               pend |= 1u << spos;
-              spos = (spos + GE) & (Lay::kStages - 1);
+              spos = (spos + GE) % Lay::kStages;
             }
           }
           __syncwarp();
@@ -691,7 +692,7 @@ __global__ void __launch_bounds__(320, 1)
               }
             }
             if (issuer) umma_commit(bempty(spos));
-            spos = (spos + GA) & (Lay::kStages - 1);
+            spos = (spos + GA) % Lay::kStages;
           } else {
             for (int dc = 0; dc < Lay::NDC; ++dc) {
               if (!(ok = mbar_wait_warp(bfull(spos), (fph >> spos) & 1u, ab))) break;
@@ -708,7 +709,7 @@ __global__ void __launch_bounds__(320, 1)
                 if (issuer) umma_f16_ts(dS, aL, dH + ko, idesc, 1u);
               }
               if (issuer) umma_commit(bempty(spos));
-              spos = (spos + GE) & (Lay::kStages - 1);
+              spos = (spos + GE) % Lay::kStages;
             }
             if (!ok) break;
           }
@@ -954,31 +955,39 @@ __global__ void __launch_bounds__(320, 1)
 template <int NB>
 __global__ void __launch_bounds__(256) block_list_kernel(const TopkParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t nrows = (int64_t)p.Hq * p.nQB;
-  const int64_t step = (int64_t)gridDim.x * 8;
-  auto load = [&](int64_t row, uint32_t (&wv)[NB], int& nb) {
-    const int i = (int)(row % p.nQB), h = (int)(row / p.nQB);
-    const int nwords = ((i >> 7) + 1) * 4;
+  const int nrows = p.Hq * p.nQB;   // below 2^31 (checked by the host)
+  const int step = (int)gridDim.x * 8;
+  // row = h * nQB + i, advanced by step without a division per row
+  const int dh = step / p.nQB, di = step % p.nQB;
+  int row = (int)blockIdx.x * 8 + warp;
+  if (row >= nrows) return;
+  int h = row / p.nQB, i = row % p.nQB;
+  auto load = [&](int hh, int ii, uint32_t (&wv)[NB], int& nb) {
+    const int nwords = ((ii >> 7) + 1) * 4;
     nb = (nwords + 31) / 32;
-    const uint32_t* mr = topk_mask_row(p.masks, p.nrt, h, i);
+    const uint32_t* mr = topk_mask_row(p.masks, p.nrt, hh, ii);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       const int w = 32 * b + lane;
       wv[b] = (b < nb && w < nwords) ? __ldcg(mr + w) : 0u;
     }
   };
-  int64_t row = (int64_t)blockIdx.x * 8 + warp;
-  if (row >= nrows) return;
   uint32_t cur[NB], nxt[NB];
   int nbc = 0, nbn = 0;
-  load(row, cur, nbc);
+  load(h, i, cur, nbc);
   for (; row < nrows; row += step) {
-    const int64_t nrow = row + step;
-    if (nrow < nrows) load(nrow, nxt, nbn);
-    topk_emit_row<NB>(p, (int)(row / p.nQB), (int)(row % p.nQB), cur, nbc, lane);
+    int hn = h + dh, in = i + di;
+    if (in >= p.nQB) {
+      in -= p.nQB;
+      ++hn;
+    }
+    if (row + step < nrows) load(hn, in, nxt, nbn);
+    topk_emit_row<NB>(p, h, i, cur, nbc, lane);
 #pragma unroll
     for (int b = 0; b < NB; ++b) cur[b] = nxt[b];
     nbc = nbn;
+    h = hn;
+    i = in;
   }
 }
 
