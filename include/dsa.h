@@ -80,8 +80,9 @@ enum {
  *             DSA_ERR_CAPACITY).
  *  pooled_k   optional [Hkv][n/64][d] fp32 out: the per-block mean keys.
  *             Required in pool-only mode.
- *  Ranking uses fp32-accurate scores (three TF32 tensor-core products of the
- *  split means, |error| ~ 2^-21 of |Q̄||K̄|); the remaining candidates of query
+ *  Ranking uses fp32-accurate scores (three FP16 tensor-core products of the
+ *  means split into hi + lo after a power-of-two scale per query block and per
+ *  KV head, |error| ~ 2^-21 of |Q̄||K̄|); the remaining candidates of query
  *  block i are blocks 1..i-1.  A bounded wait that expires sets the workspace
  *  status word (DSA_ERR_TIMEOUT through dsa_get_status).
  */
