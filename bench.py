@@ -387,7 +387,9 @@ def run_cluster_decode(args, local):
     keys (3 Lloyd rounds, timed once as the offline build), then per step every
     q-head keeps its 512 best clusters and attends over them plus the newest
     64 tokens.  GB/s counts the union of a GQA group's kept clusters' K/V rows
-    (each row is read once per (batch, KV head)), the centroids and q / o."""
+    (each row is read once per (batch, KV head)), the centroids and q / o.
+    The decode reads the context from a copy in cluster order (made once,
+    timed as pack_ms); the token-gather form is timed beside it."""
     import dynamic_sparse_attention_03_b200 as dsa
 
     dev = torch.device("cuda", local)
@@ -418,24 +420,41 @@ def run_cluster_decode(args, local):
         mask[:, h // grp] |= m2 > 0
     union_tokens = int((size * mask).sum().item()) + B * Hkv * (S - n_ctx)
     total = union_tokens * 2 * dd * 2 + B * Hkv * C * dd * 4 + 2 * B * Hq * dd * 2
-    for _ in range(3):
-        dsa.cluster_decode_attn(dw.q, dw.k_cache, dw.v_cache, cent, off, tok, n_ctx, keep, out=o, ws=ws)
+    # the context's K/V copied once in cluster order (also offline): the decode
+    # then reads each kept cluster as one contiguous range
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    packed = dsa.cluster_pack_kv(dw.k_cache, dw.v_cache, tok, n_ctx)
+    p1.record(stream)
     torch.cuda.synchronize()
-    reps = 20
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        dsa.cluster_decode_attn(dw.q, dw.k_cache, dw.v_cache, cent, off, tok, n_ctx, keep, out=o, ws=ws)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
+    pack_ms = p0.elapsed_time(p1)
+
+    def timed(pk):
+        for _ in range(3):
+            dsa.cluster_decode_attn(dw.q, dw.k_cache, dw.v_cache, cent, off, tok, n_ctx, keep, out=o, ws=ws,
+                                    packed=pk)
+        torch.cuda.synchronize()
+        reps = 20
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            dsa.cluster_decode_attn(dw.q, dw.k_cache, dw.v_cache, cent, off, tok, n_ctx, keep, out=o, ws=ws,
+                                    packed=pk)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ms = timed(packed)
+    ms_gather = timed(None)
     peaks, src = load_peaks()
     gbs = total / (ms * 1e-3) / 1e9
-    del dw
+    del dw, packed
     return {"workload": "decode-b16-128k, 2048 K-means clusters of the first S-64 keys, keep 512 + tail",
             "ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-            "bytes_per_step": total, "union_tokens": union_tokens, "kmeans_build_ms": round(build_ms, 2),
-            "kmeans_rounds": iters, "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": src}
+            "bytes_per_step": total, "union_tokens": union_tokens, "kv_layout": "cluster-ordered copy",
+            "ms_token_gather": round(ms_gather, 4), "kmeans_build_ms": round(build_ms, 2),
+            "kmeans_rounds": iters, "pack_ms": round(pack_ms, 3), "peak_hbm_gbs": peaks["hbm_gbs"],
+            "peak_source": src}
 
 
 def run_vs(args, local):

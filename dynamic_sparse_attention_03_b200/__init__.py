@@ -13,6 +13,7 @@ Entry points (same names as the C ABI):
   block_sparse_attn_fwd  causal attention over the chosen blocks and columns
   sparse_decode_attn     centroid-ranked sparse decode
   kmeans_clusters        K-means key clusters of a fixed context (centroids, cluster -> key map)
+  cluster_pack_kv        the context's K and V rows copied in cluster order
   cluster_decode_attn    decode ranked by K-means cluster centroids
 """
 
@@ -29,7 +30,7 @@ import torch
 __all__ = [
     "DSAError", "load_library", "SYMBOLS", "sparse_index_estimate", "pool_keys", "vertical_slash_index",
     "block_sparse_attn_fwd", "sparse_decode_attn", "get_status", "block_index_capacity", "Workspace",
-    "kmeans_clusters", "cluster_decode_attn",
+    "kmeans_clusters", "cluster_pack_kv", "cluster_decode_attn",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,6 +45,7 @@ SYMBOLS = (
     "sparse_decode_attn_static",
     "a_shape_index",
     "kmeans_clusters",
+    "cluster_pack_kv",
     "cluster_decode_attn",
     "dsa_get_status",
     "dsa_block_index_capacity",
@@ -81,7 +83,9 @@ _SIGS = {
     "sparse_decode_attn_static": [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P],
     "a_shape_index": [_I, _I, _I, _I, _P, _P, _I, _P],
     "kmeans_clusters": [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P],
-    "cluster_decode_attn": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P, _SZ, _P],
+    "cluster_pack_kv": [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P],
+    "cluster_decode_attn": [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P,
+                            _SZ, _P],
     "dsa_get_status": [_P, _P],
     "dsa_block_index_capacity": [_I, _I, _I, _F],
     "dsa_version": [],
@@ -371,16 +375,39 @@ def kmeans_clusters(k_cache: torch.Tensor, n_ctx: int, n_clusters: int, iters: i
     return cent, assign, offsets, tokens
 
 
+def cluster_pack_kv(k_cache: torch.Tensor, v_cache: torch.Tensor, tokens: torch.Tensor, n_ctx: int,
+                    out: Optional[tuple] = None):
+    """The first n_ctx rows of k_cache / v_cache [B][Hkv][S][d] bf16 copied in
+    cluster order (tokens from kmeans_clusters): returns (k_packed, v_packed)
+    [B][Hkv][n_ctx][d] with k_packed[b, g, p] = k_cache[b, g, tokens[b, g, p]]."""
+    _need_cuda(k_cache, v_cache, tokens)
+    _need_dtype(k_cache, torch.bfloat16, "k_cache")
+    _need_dtype(v_cache, torch.bfloat16, "v_cache")
+    B, Hkv, S, d = k_cache.shape
+    if out is None:
+        kp = torch.empty((B, Hkv, int(n_ctx), d), dtype=torch.bfloat16, device=k_cache.device)
+        vp = torch.empty_like(kp)
+    else:
+        kp, vp = out
+    _check(load_library().cluster_pack_kv(_ptr(k_cache), _ptr(v_cache), _ptr(tokens), B, Hkv, S, d, int(n_ctx),
+                                          _ptr(kp), _ptr(vp), _stream(k_cache.device)), "cluster_pack_kv")
+    return kp, vp
+
+
 def cluster_decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, centroids: torch.Tensor,
                         offsets: torch.Tensor, tokens: torch.Tensor, n_ctx: int, keep: int,
                         scale: Optional[float] = None, return_sel: bool = False,
-                        out: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None):
+                        out: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None,
+                        packed: Optional[tuple] = None):
     """Decode over K-means clusters: q [B][Hq][d], caches [B][Hkv][S][d] bf16,
     centroids / offsets / tokens from kmeans_clusters.  Each q-head keeps its
     `keep` best non-empty clusters by q.c (ties to the lower cluster) and attends
-    over their keys plus the unclustered tail [n_ctx, S).  Returns O [B][Hq][d]
-    bf16 (and sel_idx [B][Hq][keep] ascending cluster ids, sel_cnt [B][Hq])."""
-    _need_cuda(q, k_cache, v_cache, centroids, offsets, tokens, out)
+    over their keys plus the unclustered tail [n_ctx, S).  `packed` is
+    cluster_pack_kv's (k_packed, v_packed), read instead of gathering rows by
+    token id (same result).  Returns O [B][Hq][d] bf16 (and sel_idx [B][Hq][keep]
+    ascending cluster ids, sel_cnt [B][Hq])."""
+    kp, vp = packed if packed is not None else (None, None)
+    _need_cuda(q, k_cache, v_cache, centroids, offsets, tokens, out, kp, vp)
     _need_dtype(centroids, torch.float32, "centroids")
     B, Hq, d = q.shape
     Hkv, S = k_cache.shape[1], k_cache.shape[2]
@@ -392,7 +419,7 @@ def cluster_decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.T
     if return_sel:
         sel_idx = torch.empty((B, Hq, kcap), dtype=torch.int32, device=q.device)
         sel_cnt = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
-    args = [_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(centroids), _ptr(offsets), _ptr(tokens), B, Hq, Hkv, S, d,
-            int(n_ctx), C, int(keep), float(scale), _ptr(o), _ptr(sel_idx), _ptr(sel_cnt), kcap]
+    args = [_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(centroids), _ptr(offsets), _ptr(tokens), _ptr(kp), _ptr(vp),
+            B, Hq, Hkv, S, d, int(n_ctx), C, int(keep), float(scale), _ptr(o), _ptr(sel_idx), _ptr(sel_cnt), kcap]
     _call_with_ws("cluster_decode_attn", args, q.device, ws)
     return (o, sel_idx, sel_cnt) if return_sel else o

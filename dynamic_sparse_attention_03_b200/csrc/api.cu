@@ -190,10 +190,22 @@ int launch_decode(const DecodeParams& p, int B, int Hkv, int nchmax, size_t sel_
 template <int D, int G>
 int launch_cluster_decode(const ClusterParams& cp, int B, int Hkv, int nchmax, size_t sel_smem, cudaStream_t st) {
   int rc;
+  // q.c for every cluster, 64 centroids of one (batch, KV head) per CTA
+  DecodeParams sp = cp.dp;
+  sp.cent = cp.cent;
+  sp.nb = cp.C;
+  sp.scores = const_cast<float*>(cp.scores);
+  decode_score_kernel<D, G><<<dim3(B * Hkv, (cp.C + 63) / 64), 256, 0, st>>>(sp);
+  if ((rc = launch_check())) return rc;
   if ((rc = set_smem(cluster_select_kernel<D, G, 256>, sel_smem))) return rc;
   cluster_select_kernel<D, G, 256><<<B * Hkv, 256, sel_smem, st>>>(cp);
   if ((rc = launch_check())) return rc;
-  cluster_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 128, 0, st>>>(cp.dp);
+  if (cp.dp.n_packed > 0) {
+    if ((rc = set_smem(cluster_stream_attn_kernel<D, G>, ClStreamLayout<D>::kBytes))) return rc;
+    cluster_stream_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 160, ClStreamLayout<D>::kBytes, st>>>(cp.dp);
+  } else {
+    cluster_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 128, 0, st>>>(cp.dp);
+  }
   return launch_check();
 }
 
@@ -596,11 +608,33 @@ int kmeans_clusters(const void* k_cache, int B, int Hkv, int S, int d, int n_ctx
   return DSA_OK;
 }
 
+int cluster_pack_kv(const void* k_cache, const void* v_cache, const int32_t* tokens, int B, int Hkv, int S, int d,
+                    int n_ctx, void* k_packed, void* v_packed, dsa_stream_t stream) {
+  if (!k_cache || !v_cache || !tokens || !k_packed || !v_packed) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || S <= 0 || n_ctx <= 0 || n_ctx > S) return DSA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return DSA_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hkv > 65535 || (int64_t)S * d >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_packed) || !aligned16(v_packed))
+    return DSA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid((unsigned)((n_ctx + 7) / 8), (unsigned)(B * Hkv));
+  const auto* k = static_cast<const __nv_bfloat16*>(k_cache);
+  const auto* v = static_cast<const __nv_bfloat16*>(v_cache);
+  auto* kp = static_cast<__nv_bfloat16*>(k_packed);
+  auto* vp = static_cast<__nv_bfloat16*>(v_packed);
+  if (d == 128) cluster_pack_kernel<128><<<grid, 256, 0, st>>>(k, v, tokens, S, n_ctx, kp, vp);
+  else cluster_pack_kernel<64><<<grid, 256, 0, st>>>(k, v, tokens, S, n_ctx, kp, vp);
+  return launch_check();
+}
+
 int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache, const float* centroids,
-                        const int32_t* offsets, const int32_t* tokens, int B, int Hq, int Hkv, int S, int d,
-                        int n_ctx, int C, int keep, float scale, void* o, int32_t* sel_idx, int32_t* sel_cnt, int kcap,
-                        void* ws, size_t* ws_bytes, dsa_stream_t stream) {
+                        const int32_t* offsets, const int32_t* tokens, const void* k_packed, const void* v_packed,
+                        int B, int Hq, int Hkv, int S, int d, int n_ctx, int C, int keep, float scale, void* o,
+                        int32_t* sel_idx, int32_t* sel_cnt, int kcap, void* ws, size_t* ws_bytes,
+                        dsa_stream_t stream) {
   if (!q || !k_cache || !v_cache || !centroids || !offsets || !tokens || !o || !ws_bytes) return DSA_ERR_INVALID_ARG;
+  if ((k_packed == nullptr) != (v_packed == nullptr)) return DSA_ERR_INVALID_ARG;
+  if (k_packed && (!aligned16(k_packed) || !aligned16(v_packed))) return DSA_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S <= 0 || n_ctx <= 0 || n_ctx > S || C <= 0 || keep < 0)
     return DSA_ERR_INVALID_ARG;
   if (keep == 0 && n_ctx == S) return DSA_ERR_INVALID_ARG;   // nothing to attend
@@ -611,15 +645,19 @@ int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache,
   if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(centroids)) return DSA_ERR_INVALID_ARG;
   if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
   if (sel_idx && kcap < std::min(keep, C)) return DSA_ERR_CAPACITY;
-  const size_t sel_smem = (size_t)grp * d * 4 + (size_t)grp * C * 4 + (size_t)C * 12 + C;
+  const size_t sel_smem = (size_t)grp * C * 4 + (size_t)C * 12 + C;
   if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
   const int nchmax = (S + kClChunk - 1) / kClChunk;
   WsCarve c(ws);
   ClusterParams cp{};
   DecodeParams& p = cp.dp;
   p.status = static_cast<uint32_t*>(c.take(kStatusBytes));
-  p.uidx = static_cast<int32_t*>(c.take((size_t)B * Hkv * S * 4));
-  p.umask = static_cast<uint8_t*>(c.take((size_t)B * Hkv * S));
+  // union lists per (batch, KV head), rows padded to 16 entries (the head
+  // masks are bulk-copied 16-byte aligned)
+  const int lstride = (S + 15) & ~15;
+  p.uidx = static_cast<int32_t*>(c.take((size_t)B * Hkv * lstride * 4));
+  p.umask = static_cast<uint8_t*>(c.take((size_t)B * Hkv * lstride));
+  float* cl_scores = static_cast<float*>(c.take((size_t)B * Hq * C * 4));
   p.ucnt = static_cast<int32_t*>(c.take((size_t)B * Hkv * 4));
   p.part_ml = static_cast<float*>(c.take((size_t)B * Hq * nchmax * 2 * 4));
   p.part_acc = static_cast<float*>(c.take((size_t)B * Hq * nchmax * d * 4));
@@ -638,7 +676,7 @@ int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache,
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.S = S;
-  p.nb = S;
+  p.nb = lstride;   // list row stride
   p.grp = grp;
   p.keep = keep;
   p.kcap = kcap;
@@ -647,8 +685,12 @@ int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache,
   cp.cent = centroids;
   cp.off = offsets;
   cp.tok = tokens;
+  cp.scores = cl_scores;
   cp.C = C;
   cp.n_ctx = n_ctx;
+  p.kp = static_cast<const __nv_bfloat16*>(k_packed);
+  p.vp = static_cast<const __nv_bfloat16*>(v_packed);
+  p.n_packed = k_packed ? n_ctx : 0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int rc;
   switch (grp * 1000 + d) {

@@ -20,13 +20,16 @@
 // Lloyd rounds run (assign, csr, update) `iters` times.
 //
 // Online decode:
-//  cluster_select_kernel: per (batch, KV head): q.c for the group's q-heads
-//                        over the non-empty clusters, the top `keep` per head
+//  cluster_select_kernel: per (batch, KV head): the scores of the non-empty
+//                        clusters (q.c for every cluster comes from
+//                        decode_score_kernel, many CTAs), the top `keep` per head
 //                        (ties to the lower cluster), and the union of the
 //                        group's kept clusters flattened into one token list
 //                        with a per-token head mask, followed by the
 //                        unclustered tail [n_ctx, S) that every head attends.
-//  cluster_attn_kernel:  2048 tokens of the union list per CTA: K and V rows
+//  cluster_attn_kernel:  kClChunk entries of the union list per CTA: K and V rows
+//                        read by position from the cluster-ordered copy
+//                        (cluster_pack_kernel) when there is one, else
 //                        gathered by token id (16-byte loads, each row read
 //                        once for the whole GQA group), an online softmax per
 //                        head with the token's head mask, one partial per
@@ -312,6 +315,7 @@ struct ClusterParams {
   const float* cent;        // [BG][C][D]
   const int32_t* off;       // [BG][C + 1]
   const int32_t* tok;       // [BG][n_ctx]
+  const float* scores;      // [B * Hq][C] q.c of every cluster (decode_score_kernel)
   int C, n_ctx;
 };
 
@@ -323,17 +327,12 @@ __global__ void __launch_bounds__(NT) cluster_select_kernel(const ClusterParams 
   const int bg = blockIdx.x;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int C = cp.C;
-  float* qf = reinterpret_cast<float*>(csm);                        // [GRP][D]
-  float* sc = qf + GRP * D;                                          // [GRP][C] (compacted candidates)
+  float* sc = reinterpret_cast<float*>(csm);                        // [GRP][C] (compacted candidates)
   int32_t* cand = reinterpret_cast<int32_t*>(sc + (size_t)GRP * C);  // [C] non-empty cluster ids
   int32_t* tmp = cand + C;                                           // [C]
   int32_t* ubase = tmp + C;                                          // [C] union token offsets
   uint8_t* mask = reinterpret_cast<uint8_t*>(ubase + C);             // [C]
   const int32_t* off = cp.off + (size_t)bg * (C + 1);
-  for (int x = threadIdx.x; x < GRP * D; x += NT) {
-    const int hh = x / D, c = x % D;
-    qf[x] = __bfloat162float(p.q[((size_t)b * p.Hq + g * GRP + hh) * D + c]);
-  }
   // non-empty clusters, ascending (block scan over per-thread ranges)
   const int per = (C + NT - 1) / NT;
   const int c0 = min(C, (int)threadIdx.x * per), c1 = min(C, c0 + per);
@@ -347,29 +346,12 @@ __global__ void __launch_bounds__(NT) cluster_select_kernel(const ClusterParams 
   for (int c = c0; c < c1; ++c)
     if (off[c + 1] > off[c]) cand[pos++] = c;
   __syncthreads();
-  // scores: one warp per candidate centroid, lanes over d
-  constexpr int PER = D / 32;
+  // the candidates' scores, computed for every cluster by decode_score_kernel
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float qreg[GRP][PER];
-#pragma unroll
-  for (int hh = 0; hh < GRP; ++hh)
-#pragma unroll
-    for (int a = 0; a < PER; ++a) qreg[hh][a] = qf[hh * D + lane * PER + a];
-  const float* crow = cp.cent + (size_t)bg * C * D;
-  for (int x = warp; x < ncand; x += NT / 32) {
-    const int c = cand[x];
-    float cv[PER];
-#pragma unroll
-    for (int a = 0; a < PER; ++a) cv[a] = __ldg(crow + (size_t)c * D + lane * PER + a);
-#pragma unroll
-    for (int hh = 0; hh < GRP; ++hh) {
-      float s = 0.f;
-#pragma unroll
-      for (int a = 0; a < PER; ++a) s = fmaf(qreg[hh][a], cv[a], s);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-      if (lane == 0) sc[(size_t)hh * C + x] = s;
-    }
+  const float* gsc = cp.scores + ((size_t)b * p.Hq + g * GRP) * C;   // the group's rows are contiguous
+  for (int x = threadIdx.x; x < GRP * ncand; x += NT) {
+    const int hh = x / ncand, y = x % ncand;
+    sc[(size_t)hh * C + y] = gsc[(size_t)hh * C + cand[y]];
   }
   __syncthreads();
   const int e = min(p.keep, ncand);
@@ -395,14 +377,15 @@ __global__ void __launch_bounds__(NT) cluster_select_kernel(const ClusterParams 
     if (mask[c]) ub += off[c + 1] - off[c];
   }
   __syncthreads();
-  int32_t* ui = p.uidx + (size_t)bg * p.S;
-  uint8_t* um = p.umask + (size_t)bg * p.S;
+  int32_t* ui = p.uidx + (size_t)bg * p.nb;
+  uint8_t* um = p.umask + (size_t)bg * p.nb;
   const int32_t* tk = cp.tok + (size_t)bg * cp.n_ctx;
+  const bool packed = p.n_packed > 0;   // positions in the cluster-ordered copy, else token ids
   for (int x = warp; x < C; x += NT / 32) {
     if (!mask[x]) continue;
     const int a = off[x], n = off[x + 1] - a, dst = ubase[x];
     for (int y = lane; y < n; y += 32) {
-      ui[dst + y] = tk[a + y];
+      ui[dst + y] = packed ? a + y : tk[a + y];
       um[dst + y] = mask[x];
     }
   }
@@ -422,7 +405,7 @@ __global__ void __launch_bounds__(NT) cluster_select_kernel(const ClusterParams 
 // 8 q-heads per KV head to bound registers), lane % 16 owns D / 16 dims; rows
 // are gathered straight from global memory with 16-byte (8-byte at D = 64)
 // loads, and an online softmax per (lane, head) runs over the whole chunk.
-constexpr int kClChunk = 2048;
+constexpr int kClChunk = 4096;
 
 template <int D, int GRP>
 __global__ void __launch_bounds__(128) cluster_attn_kernel(const DecodeParams p) {
@@ -436,8 +419,8 @@ __global__ void __launch_bounds__(128) cluster_attn_kernel(const DecodeParams p)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int DPL = D / 16;
   const int half = lane >> 4, dl = lane & 15;
-  const int32_t* ui = p.uidx + (size_t)bg * p.S;
-  const uint8_t* um = p.umask + (size_t)bg * p.S;
+  const int32_t* ui = p.uidx + (size_t)bg * p.nb;
+  const uint8_t* um = p.umask + (size_t)bg * p.nb;
   const size_t head_base = (size_t)bg * p.S * D;
   float qv[GRP][DPL];
 #pragma unroll
@@ -469,10 +452,15 @@ __global__ void __launch_bounds__(128) cluster_attn_kernel(const DecodeParams p)
       }
       if (u < c1) {
         msk[it] = um[u];
-        const size_t row = head_base + (size_t)ui[u] * D + dl * DPL;
+        // entries below n_packed index the cluster-ordered copy, the rest the cache
+        const int idx = ui[u];
+        const bool pk = idx < p.n_packed;
+        const size_t row = (pk ? ((size_t)bg * p.n_packed + idx) * D : head_base + (size_t)idx * D) + dl * DPL;
+        const __nv_bfloat16* kb = pk ? p.kp : p.kc;
+        const __nv_bfloat16* vb = pk ? p.vp : p.vc;
         if (DPL == 8) {
-          const uint4 kr = __ldg(reinterpret_cast<const uint4*>(p.kc + row));
-          const uint4 vr = __ldg(reinterpret_cast<const uint4*>(p.vc + row));
+          const uint4 kr = __ldg(reinterpret_cast<const uint4*>(kb + row));
+          const uint4 vr = __ldg(reinterpret_cast<const uint4*>(vb + row));
           const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
           const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
 #pragma unroll
@@ -484,8 +472,8 @@ __global__ void __launch_bounds__(128) cluster_attn_kernel(const DecodeParams p)
             vf[it][(2 * a + 1) % DPL] = vv.y;
           }
         } else {
-          const uint2 kr = __ldg(reinterpret_cast<const uint2*>(p.kc + row));
-          const uint2 vr = __ldg(reinterpret_cast<const uint2*>(p.vc + row));
+          const uint2 kr = __ldg(reinterpret_cast<const uint2*>(kb + row));
+          const uint2 vr = __ldg(reinterpret_cast<const uint2*>(vb + row));
           const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
           const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
 #pragma unroll
@@ -567,6 +555,279 @@ __global__ void __launch_bounds__(128) cluster_attn_kernel(const DecodeParams p)
       p.part_ml[(ph * p.nchmax + chunk) * 2 + 0] = M;
       p.part_ml[(ph * p.nchmax + chunk) * 2 + 1] = L;
     }
+  }
+}
+
+// ---------------------------------------------------------------- decode: streamed union
+// With the cluster-ordered copy, the union list is a few long runs of
+// consecutive rows (kept clusters, then the tail), so it streams like the
+// block decode: per CTA kClChunk entries in units of 64; the producer warp
+// finds the runs of a unit (ballots over consecutive positions) and lane 0
+// bulk-copies each run's K and V rows into a ring stage (one copy per run and
+// operand, the stage's byte count expected up front); four consumer warps
+// score the unit's rows for the group's q-heads with each row's head mask
+// and keep an online softmax per (warp, head), as decode_attn_kernel does.
+template <int D>
+struct ClStreamLayout : DecLayout<D> {
+  static constexpr int kMask = (DecLayout<D>::kBytes + 15) & ~15;   // 64 head-mask bytes per stage
+  static constexpr int kBytes = kMask + kDecStages * 64;
+};
+
+template <int D, int GRP>
+__global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const DecodeParams p) {
+  using Lay = ClStreamLayout<D>;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const uint32_t sb = smem_u32(dsm);
+  const int bg = blockIdx.x, chunk = blockIdx.y;
+  const int cnt = p.ucnt[bg];
+  const int e0 = chunk * kClChunk;
+  if (e0 >= cnt || status_timed_out(p.status)) return;
+  const int e1 = min(cnt, e0 + kClChunk);
+  const int nu = (e1 - e0 + 63) / 64;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar0 = sb + Lay::kBar;
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (kDecStages + s); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + Lay::kBar + 2 * kDecStages * 8);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const AbortState ab{abort_flag, p.status};
+  const int32_t* ui = p.uidx + (size_t)bg * p.nb;
+  const uint8_t* um = p.umask + (size_t)bg * p.nb;
+  constexpr uint32_t kRowBytes = D * 2;
+
+  if (warp == 4) {
+    // producer warp: runs of consecutive positions of each unit
+    int u = 0;
+    for (; u < nu; ++u) {
+      const int s = u % kDecStages;
+      if (u >= kDecStages && !mbar_wait_warp(empty(s), ((u / kDecStages) - 1) & 1, ab)) break;
+      const int rb = e0 + 64 * u, rows = min(64, e1 - rb);
+      const int pa = lane < rows ? ui[rb + lane] : -1;
+      const int pb = lane + 32 < rows ? ui[rb + lane + 32] : -1;
+      const int up_a = __shfl_up_sync(0xFFFFFFFFu, pa, 1), last_a = __shfl_sync(0xFFFFFFFFu, pa, 31);
+      const int up_b = __shfl_up_sync(0xFFFFFFFFu, pb, 1);
+      const int prev_b = lane == 0 ? last_a : up_b;
+      // a run starts at row 0, after a gap, and where the cache tail begins
+      // (positions below n_packed are in the copy, the rest in the cache)
+      const bool st_a = lane < rows && (lane == 0 || pa != up_a + 1 || pa == p.n_packed);
+      const bool st_b = lane + 32 < rows && (pb != prev_b + 1 || pb == p.n_packed);
+      uint64_t starts = (uint64_t)__ballot_sync(0xFFFFFFFFu, st_a) | ((uint64_t)__ballot_sync(0xFFFFFFFFu, st_b) << 32);
+      // the unit's head masks ride with its rows (64 bytes, 16-byte aligned)
+      const uint32_t mbytes = (uint32_t)((rows + 15) & ~15);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(full(s), (uint32_t)rows * 2u * kRowBytes + mbytes);
+        bulk_load(sb + Lay::kMask + s * 64, um + rb, mbytes, full(s));
+      }
+      while (starts) {   // warp-uniform
+        const int r = __ffsll((long long)starts) - 1;
+        starts &= starts - 1ull;
+        const int rn = starts ? __ffsll((long long)starts) - 1 : rows;
+        const int pos = __shfl_sync(0xFFFFFFFFu, r < 32 ? pa : pb, r & 31);
+        if (lane == 0) {
+          const bool pk = pos < p.n_packed;
+          const size_t src = (pk ? (size_t)bg * p.n_packed : (size_t)bg * p.S) * D + (size_t)pos * D;
+          const uint32_t bytes = (uint32_t)(rn - r) * kRowBytes;
+          const uint32_t dst = sb + s * Lay::kStage + (uint32_t)r * kRowBytes;
+          bulk_load(dst, (pk ? p.kp : p.kc) + src, bytes, full(s));
+          bulk_load(dst + Lay::kBlkBytes, (pk ? p.vp : p.vc) + src, bytes, full(s));
+        }
+      }
+      __syncwarp();
+    }
+    if (lane == 0)
+      for (int w = max(0, u - kDecStages); w < u; ++w)
+        mbar_wait_cleanup(full(w % kDecStages), (w / kDecStages) & 1, 200000000ull);
+    return;
+  }
+  // consumers: warp w takes rows 16w .. 16w+15 of every unit; the two half
+  // warps take alternate rows, lane%16 owns dims [DPL*(lane%16), +DPL)
+  constexpr int DPL = D / 16;
+  const int half = lane >> 4, dl = lane & 15;
+  float qv[GRP][DPL];
+#pragma unroll
+  for (int hh = 0; hh < GRP; ++hh)
+#pragma unroll
+    for (int a = 0; a < DPL; ++a)
+      qv[hh][a] = __bfloat162float(p.q[((size_t)b * p.Hq + g * GRP + hh) * D + dl * DPL + a]) * p.scale_log2;
+  float m[GRP], l[GRP], acc[GRP][DPL];
+#pragma unroll
+  for (int hh = 0; hh < GRP; ++hh) {
+    m[hh] = -INFINITY;
+    l[hh] = 0.f;
+#pragma unroll
+    for (int a = 0; a < DPL; ++a) acc[hh][a] = 0.f;
+  }
+  bool ok = true;
+  for (int u = 0; u < nu; ++u) {
+    const int s = u % kDecStages;
+    const int rb = e0 + 64 * u, rows = min(64, e1 - rb);
+    if (!mbar_wait_warp(full(s), (u / kDecStages) & 1, ab)) {
+      ok = false;
+      break;
+    }
+    const uint8_t* ms = dsm + Lay::kMask + s * 64;
+    uint32_t msk[8];
+    uint32_t mor = 0u;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int key = 16 * warp + 2 * it + half;
+      msk[it] = key < rows ? (uint32_t)ms[key] : 0u;
+      mor |= msk[it];
+    }
+    mor = __reduce_or_sync(0xFFFFFFFFu, mor);
+    const uint8_t* kb = dsm + s * Lay::kStage;
+    const uint8_t* vb = kb + Lay::kBlkBytes;
+    float kf[8][DPL], vf[8][DPL];
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int key = 16 * warp + 2 * it + half;
+      const bool valid = key < rows;   // rows past the unit's end hold stale bytes: never used
+#pragma unroll
+      for (int a = 0; a < DPL; ++a) {
+        kf[it][a] = 0.f;
+        vf[it][a] = 0.f;
+      }
+      if (valid) {
+        if constexpr (DPL == 8) {
+          const uint4 kr = *reinterpret_cast<const uint4*>(kb + key * kRowBytes + dl * 16);
+          const uint4 vr = *reinterpret_cast<const uint4*>(vb + key * kRowBytes + dl * 16);
+          const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+          const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            const float2 kk = __bfloat1622float2(k2[a]), vv = __bfloat1622float2(v2[a]);
+            kf[it][2 * a] = kk.x;
+            kf[it][2 * a + 1] = kk.y;
+            vf[it][2 * a] = vv.x;
+            vf[it][2 * a + 1] = vv.y;
+          }
+        } else {
+          const uint2 kr = *reinterpret_cast<const uint2*>(kb + key * kRowBytes + dl * 8);
+          const uint2 vr = *reinterpret_cast<const uint2*>(vb + key * kRowBytes + dl * 8);
+          const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+          const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            const float2 kk = __bfloat1622float2(k2[a]), vv = __bfloat1622float2(v2[a]);
+            kf[it][(2 * a) % DPL] = kk.x;
+            kf[it][(2 * a + 1) % DPL] = kk.y;
+            vf[it][(2 * a) % DPL] = vv.x;
+            vf[it][(2 * a + 1) % DPL] = vv.y;
+          }
+        }
+      }
+    }
+    // release the stage once every warp has its registers
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty(s));
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) {
+      if (!((mor >> hh) & 1u)) continue;   // no row of the unit kept by this head (warp-uniform)
+      float sc[8];
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        float d0 = 0.f;
+#pragma unroll
+        for (int a = 0; a < DPL; ++a) d0 = fmaf(qv[hh][a], kf[it][a], d0);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) d0 += __shfl_xor_sync(0xFFFFFFFFu, d0, o);
+        sc[it] = ((msk[it] >> hh) & 1u) ? d0 : -INFINITY;
+      }
+      float mb = sc[0];
+#pragma unroll
+      for (int it = 1; it < 8; ++it) mb = fmaxf(mb, sc[it]);
+      mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 16));
+      const float mn = fmaxf(m[hh], mb);
+      if (mn == -INFINITY) continue;   // nothing of this head in this warp yet (warp-uniform)
+      const float alpha = ex2_approx(m[hh] - mn);   // m = -inf -> 0
+      float ls = 0.f;
+#pragma unroll
+      for (int a = 0; a < DPL; ++a) acc[hh][a] *= alpha;
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const float pe = ex2_approx(sc[it] - mn);   // -inf -> 0
+        ls += pe;
+#pragma unroll
+        for (int a = 0; a < DPL; ++a) acc[hh][a] = fmaf(pe, vf[it][a], acc[hh][a]);
+      }
+      l[hh] = l[hh] * alpha + ls;
+      m[hh] = mn;
+    }
+  }
+  // merge the two half-warps (same dims, same running max), then the 4 warps
+  float* red = reinterpret_cast<float*>(dsm + Lay::kRed);   // [warp][hh][D + 2]
+#pragma unroll
+  for (int hh = 0; hh < GRP; ++hh) {
+    l[hh] += __shfl_xor_sync(0xFFFFFFFFu, l[hh], 16);
+#pragma unroll
+    for (int a = 0; a < DPL; ++a) acc[hh][a] += __shfl_xor_sync(0xFFFFFFFFu, acc[hh][a], 16);
+    float* r = red + ((size_t)warp * kMaxGrp + hh) * (D + 2);
+    if (half == 0) {
+#pragma unroll
+      for (int a = 0; a < DPL; ++a) r[dl * DPL + a] = acc[hh][a];
+    }
+    if (lane == 0) {
+      r[D] = m[hh];
+      r[D + 1] = l[hh];
+    }
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (!ok) return;
+  for (int x = threadIdx.x; x < GRP * D; x += 128) {
+    const int hh = x / D, c = x % D;
+    float M = -INFINITY;
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, red[((size_t)w * kMaxGrp + hh) * (D + 2) + D]);
+    float a = 0.f, L = 0.f;
+    if (M != -INFINITY) {
+      for (int w = 0; w < 4; ++w) {
+        const float* r = red + ((size_t)w * kMaxGrp + hh) * (D + 2);
+        if (r[D] == -INFINITY) continue;
+        const float wgt = ex2_approx(r[D] - M);
+        a += wgt * r[c];
+        L += wgt * r[D + 1];
+      }
+    }
+    const size_t ph = (size_t)b * p.Hq + g * GRP + hh;
+    p.part_acc[(ph * p.nchmax + chunk) * D + c] = a;
+    if (c == 0) {
+      p.part_ml[(ph * p.nchmax + chunk) * 2 + 0] = M;
+      p.part_ml[(ph * p.nchmax + chunk) * 2 + 1] = L;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- cluster-ordered copy
+// kp[bg][pos] = k[bg][tokens[bg][pos]] (and v) for pos < n_ctx: one warp per
+// position, lanes 0-15 copy the K row and lanes 16-31 the V row (16-byte
+// vectors at D = 128, 8-byte at D = 64); the reads gather rows, the writes
+// stream.  Done once per fixed context, so the decode reads each kept
+// cluster as one contiguous range.
+template <int D>
+__global__ void __launch_bounds__(256) cluster_pack_kernel(const __nv_bfloat16* __restrict__ k,
+                                                           const __nv_bfloat16* __restrict__ v,
+                                                           const int32_t* __restrict__ tok, int S, int n_ctx,
+                                                           __nv_bfloat16* __restrict__ kp,
+                                                           __nv_bfloat16* __restrict__ vp) {
+  const int bg = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pos = blockIdx.x * 8 + warp;
+  if (pos >= n_ctx) return;
+  const int t = tok[(size_t)bg * n_ctx + pos];
+  const int half = lane >> 4, l16 = lane & 15;
+  const __nv_bfloat16* src = (half ? v : k) + ((size_t)bg * S + t) * D;
+  __nv_bfloat16* dst = (half ? vp : kp) + ((size_t)bg * n_ctx + pos) * D;
+  if constexpr (D == 128) {
+    reinterpret_cast<uint4*>(dst)[l16] = __ldg(reinterpret_cast<const uint4*>(src) + l16);
+  } else {
+    reinterpret_cast<uint2*>(dst)[l16] = __ldg(reinterpret_cast<const uint2*>(src) + l16);
   }
 }
 

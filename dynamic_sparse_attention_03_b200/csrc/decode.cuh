@@ -46,6 +46,9 @@ struct DecodeParams {
   float* part_ml;              // ws [B*Hq][nchmax][2]
   float* part_acc;             // ws [B*Hq][nchmax][D]
   float* scores;               // ws [B*Hq][nb] q·c
+  const __nv_bfloat16* kp;     // optional [B][Hkv][n_packed][D]: K rows in cluster order
+  const __nv_bfloat16* vp;     //   (list entries below n_packed are positions in these)
+  int n_packed;                // 0 when the list holds cache token ids only
   uint32_t* status;
   int B, Hq, Hkv, S, nb, grp, keep, force_last, kcap, nchmax;
   float scale_log2;

@@ -222,6 +222,21 @@ int kmeans_clusters(const void* k_cache, int B, int Hkv, int S, int d, int n_ctx
                     size_t* ws_bytes, dsa_stream_t stream);
 
 /*
+ * cluster_pack_kv -- a copy of the fixed context's K and V rows in cluster
+ * order, made once after kmeans_clusters (Squeezed Attention, technical
+ * approach: the context is fixed, so what is computed offline is reused by
+ * every decode step): k_packed[b][g][p] = k_cache[b][g][tokens[b][g][p]] for
+ * p < n_ctx, and the same for V, so cluster c occupies positions
+ * offsets[c] .. offsets[c+1] - 1.
+ *
+ *  k_cache, v_cache  [B][Hkv][S][d] bf16.   tokens: kmeans_clusters' output.
+ *  k_packed, v_packed  [B][Hkv][n_ctx][d] bf16 out (caller-owned, 16-byte aligned).
+ * Launches one kernel on `stream`; no workspace.
+ */
+int cluster_pack_kv(const void* k_cache, const void* v_cache, const int32_t* tokens, int B, int Hkv, int S, int d,
+                    int n_ctx, void* k_packed, void* v_packed, dsa_stream_t stream);
+
+/*
  * cluster_decode_attn -- the online stage over K-means clusters (Squeezed
  * Attention, technical approach: compare the query with every centroid, keep
  * the top clusters, attend only over the keys and values of those clusters).
@@ -233,15 +248,20 @@ int kmeans_clusters(const void* k_cache, int B, int Hkv, int S, int d, int n_ctx
  *  q          [B][Hq][d] bf16.   k_cache, v_cache [B][Hkv][S][d] bf16.
  *  centroids, offsets, tokens: kmeans_clusters' outputs for the same cache.
  *  o          [B][Hq][d] bf16 out.
+ *  k_packed, v_packed  optional (both or neither) [B][Hkv][n_ctx][d] bf16:
+ *             cluster_pack_kv's cluster-ordered copy of the context.  With
+ *             it, a kept cluster is read as one contiguous range; without,
+ *             its K and V rows are gathered from the caches by token id.
  *  sel_idx    optional [B][Hq][kcap] int32 out (ascending kept clusters, -1
  *             padded), sel_cnt optional [B][Hq]; kcap >= min(keep, C).
- * K and V rows are gathered by token id; the union of a GQA group's kept
- * clusters is read once for the group.
+ * The union of a GQA group's kept clusters is read once for the group.  The
+ * result does not depend on the copy (same rows, same order).
  */
 int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache, const float* centroids,
-                        const int32_t* offsets, const int32_t* tokens, int B, int Hq, int Hkv, int S, int d,
-                        int n_ctx, int C, int keep, float scale, void* o, int32_t* sel_idx, int32_t* sel_cnt,
-                        int kcap, void* ws, size_t* ws_bytes, dsa_stream_t stream);
+                        const int32_t* offsets, const int32_t* tokens, const void* k_packed, const void* v_packed,
+                        int B, int Hq, int Hkv, int S, int d, int n_ctx, int C, int keep, float scale, void* o,
+                        int32_t* sel_idx, int32_t* sel_cnt, int kcap, void* ws, size_t* ws_bytes,
+                        dsa_stream_t stream);
 
 /*
  * dsa_get_status -- synchronize `stream`, read the workspace's device status

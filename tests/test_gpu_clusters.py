@@ -110,13 +110,18 @@ def test_kmeans_rounds_are_self_consistent():
         assert oracle.kmeans_objective(keys, cg, a) <= obj0 * (1 + 1e-6)
 
 
+@pytest.mark.parametrize("packed", [False, True])
 @pytest.mark.parametrize("B,Hq,Hkv,S,d,n_ctx,C,keep", [(2, 8, 2, 4096, 128, 4032, 64, 16),
                                                       (1, 4, 4, 2048, 64, 2048, 32, 8),
                                                       (1, 8, 1, 3072, 128, 2944, 48, 48)])
-def test_cluster_decode_matches_oracle(B, Hq, Hkv, S, d, n_ctx, C, keep):
+def test_cluster_decode_matches_oracle(B, Hq, Hkv, S, d, n_ctx, C, keep, packed):
+    """Both forms of the decode: rows gathered by token id, and rows streamed
+    from the cluster-ordered copy."""
     w = synth.make_decode("decode-b16-128k", device=DEV, B=B, S=S, Hq=Hq, Hkv=Hkv, d=d, seed=C + keep)
     cent, assign, off, tok = dsa.kmeans_clusters(w.k_cache, n_ctx, C, iters=2)
-    o, si, sc = dsa.cluster_decode_attn(w.q, w.k_cache, w.v_cache, cent, off, tok, n_ctx, keep, return_sel=True)
+    pk = dsa.cluster_pack_kv(w.k_cache, w.v_cache, tok, n_ctx) if packed else None
+    o, si, sc = dsa.cluster_decode_attn(w.q, w.k_cache, w.v_cache, cent, off, tok, n_ctx, keep, return_sel=True,
+                                        packed=pk)
     torch.cuda.synchronize()
     assert dsa.get_status() == 0
     q64, k64, v64 = f64(w.q), f64(w.k_cache), f64(w.v_cache)
@@ -153,6 +158,39 @@ def test_cluster_decode_keep_all_equals_dense():
     assert err.max().item() < 2e-2 and err.mean().item() < 2e-3
 
 
+def test_cluster_pack_kv_is_the_cluster_order_gather():
+    B, Hkv, S, d, n_ctx, C = 2, 2, 2048, 128, 1984, 32
+    w = synth.make_decode("decode-b16-128k", device=DEV, B=B, S=S, Hq=Hkv, Hkv=Hkv, d=d, seed=11)
+    _, _, _, tok = dsa.kmeans_clusters(w.k_cache, n_ctx, C, iters=2)
+    kp, vp = dsa.cluster_pack_kv(w.k_cache, w.v_cache, tok, n_ctx)
+    idx = tok.long()[..., None].expand(B, Hkv, n_ctx, d)
+    assert torch.equal(kp, torch.gather(w.k_cache, 2, idx))
+    assert torch.equal(vp, torch.gather(w.v_cache, 2, idx))
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,S,d,n_ctx,C,keep", [(2, 8, 2, 4096, 128, 4032, 64, 16),
+                                                      (1, 4, 4, 2048, 64, 2048, 32, 8),
+                                                      (1, 8, 1, 3072, 128, 2944, 48, 48)])
+def test_packed_cluster_decode_equals_gathered(B, Hq, Hkv, S, d, n_ctx, C, keep):
+    """The cluster-ordered copy holds the same rows in the same order as the
+    token gather, and both kernels give each lane the same rows when a KV head
+    has at most 4 q-heads: the outputs are then identical bit for bit (with 8
+    the gather kernel takes 4 rows per lane and sums in another order)."""
+    w = synth.make_decode("decode-b16-128k", device=DEV, B=B, S=S, Hq=Hq, Hkv=Hkv, d=d, seed=C + keep + 1)
+    cent, _, off, tok = dsa.kmeans_clusters(w.k_cache, n_ctx, C, iters=2)
+    packed = dsa.cluster_pack_kv(w.k_cache, w.v_cache, tok, n_ctx)
+    o1, si1, sc1 = dsa.cluster_decode_attn(w.q, w.k_cache, w.v_cache, cent, off, tok, n_ctx, keep, return_sel=True)
+    o2, si2, sc2 = dsa.cluster_decode_attn(w.q, w.k_cache, w.v_cache, cent, off, tok, n_ctx, keep, return_sel=True,
+                                           packed=packed)
+    torch.cuda.synchronize()
+    assert dsa.get_status() == 0
+    assert torch.equal(si1, si2) and torch.equal(sc1, sc2)
+    if Hq // Hkv <= 4:
+        assert torch.equal(o1, o2)
+    else:
+        assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
+
+
 def test_cluster_abi_rejects_bad_arguments():
     kc = torch.zeros((1, 1, 256, 128), dtype=torch.bfloat16, device=DEV)
     with pytest.raises(dsa.DSAError):
@@ -161,3 +199,6 @@ def test_cluster_abi_rejects_bad_arguments():
         dsa.kmeans_clusters(kc, 300, 8, iters=1)        # context past the cache
     with pytest.raises(dsa.DSAError):
         dsa.kmeans_clusters(kc, 256, 8, iters=0)
+    tok = torch.zeros((1, 1, 256), dtype=torch.int32, device=DEV)
+    with pytest.raises(dsa.DSAError):
+        dsa.cluster_pack_kv(kc, kc, tok, 300)          # context past the cache
