@@ -202,7 +202,8 @@ int launch_cluster_decode(const ClusterParams& cp, int B, int Hkv, int nchmax, s
   if ((rc = launch_check())) return rc;
   if (cp.dp.n_packed > 0) {
     if ((rc = set_smem(cluster_stream_attn_kernel<D, G>, ClStreamLayout<D>::kBytes))) return rc;
-    cluster_stream_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 160, ClStreamLayout<D>::kBytes, st>>>(cp.dp);
+    cluster_stream_attn_kernel<D, G>
+        <<<dim3(B * Hkv, nchmax), (kClWarps + 1) * 32, ClStreamLayout<D>::kBytes, st>>>(cp.dp);
   } else {
     cluster_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 128, 0, st>>>(cp.dp);
   }

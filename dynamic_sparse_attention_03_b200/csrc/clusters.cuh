@@ -564,18 +564,29 @@ __global__ void __launch_bounds__(128) cluster_attn_kernel(const DecodeParams p)
 // block decode: per CTA kClChunk entries in units of 64; the producer warp
 // finds the runs of a unit (ballots over consecutive positions) and lane 0
 // bulk-copies each run's K and V rows into a ring stage (one copy per run and
-// operand, the stage's byte count expected up front); four consumer warps
+// operand, the stage's byte count expected up front); the consumer warps
 // score the unit's rows for the group's q-heads with each row's head mask
-// and keep an online softmax per (warp, head), as decode_attn_kernel does.
+// and keep an online softmax per (warp, head), as decode_attn_kernel does,
+// but eight of them with four rows per lane (fewer registers, two warps per
+// scheduler, and a head is skipped for any 8-row slice none of whose rows it
+// kept).
+constexpr int kClWarps = 8;   // consumer warps: 8 rows of each unit per warp, 4 per lane
+
 template <int D>
-struct ClStreamLayout : DecLayout<D> {
-  static constexpr int kMask = (DecLayout<D>::kBytes + 15) & ~15;   // 64 head-mask bytes per stage
-  static constexpr int kBytes = kMask + kDecStages * 64;
+struct ClStreamLayout {
+  static constexpr int kBlkBytes = 64 * D * 2;                  // 64 K (or V) rows
+  static constexpr int kStage = 2 * kBlkBytes;
+  static constexpr int kRed = kDecStages * kStage;              // warp partials [warp][head][D + 2]
+  static constexpr int kRedBytes = kClWarps * kMaxGrp * (D + 2) * 4;
+  static constexpr int kMask = kRed + kRedBytes;                // 64 head-mask bytes per stage
+  static constexpr int kBar = kMask + kDecStages * 64;
+  static constexpr int kBytes = kBar + 2 * kDecStages * 8 + 16;
 };
 
 template <int D, int GRP>
-__global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__((kClWarps + 1) * 32, 1) cluster_stream_attn_kernel(const DecodeParams p) {
   using Lay = ClStreamLayout<D>;
+  constexpr int NW = kClWarps, TPL = 32 / NW;   // rows per lane per unit
   extern __shared__ __align__(16) uint8_t dsm[];
   const uint32_t sb = smem_u32(dsm);
   const int bg = blockIdx.x, chunk = blockIdx.y;
@@ -593,7 +604,7 @@ __global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const Decod
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), 4);
+      mbar_init(empty(s), NW);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -604,7 +615,7 @@ __global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const Decod
   const uint8_t* um = p.umask + (size_t)bg * p.nb;
   constexpr uint32_t kRowBytes = D * 2;
 
-  if (warp == 4) {
+  if (warp == NW) {
     // producer warp: runs of consecutive positions of each unit
     int u = 0;
     for (; u < nu; ++u) {
@@ -648,7 +659,7 @@ __global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const Decod
         mbar_wait_cleanup(full(w % kDecStages), (w / kDecStages) & 1, 200000000ull);
     return;
   }
-  // consumers: warp w takes rows 16w .. 16w+15 of every unit; the two half
+  // consumers: warp w takes rows 2 TPL w .. of every unit; the two half
   // warps take alternate rows, lane%16 owns dims [DPL*(lane%16), +DPL)
   constexpr int DPL = D / 16;
   const int half = lane >> 4, dl = lane & 15;
@@ -675,21 +686,21 @@ __global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const Decod
       break;
     }
     const uint8_t* ms = dsm + Lay::kMask + s * 64;
-    uint32_t msk[8];
+    uint32_t msk[TPL];
     uint32_t mor = 0u;
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int key = 16 * warp + 2 * it + half;
+    for (int it = 0; it < TPL; ++it) {
+      const int key = 2 * TPL * warp + 2 * it + half;
       msk[it] = key < rows ? (uint32_t)ms[key] : 0u;
       mor |= msk[it];
     }
     mor = __reduce_or_sync(0xFFFFFFFFu, mor);
     const uint8_t* kb = dsm + s * Lay::kStage;
     const uint8_t* vb = kb + Lay::kBlkBytes;
-    float kf[8][DPL], vf[8][DPL];
+    float kf[TPL][DPL], vf[TPL][DPL];
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int key = 16 * warp + 2 * it + half;
+    for (int it = 0; it < TPL; ++it) {
+      const int key = 2 * TPL * warp + 2 * it + half;
       const bool valid = key < rows;   // rows past the unit's end hold stale bytes: never used
 #pragma unroll
       for (int a = 0; a < DPL; ++a) {
@@ -732,9 +743,9 @@ __global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const Decod
 #pragma unroll
     for (int hh = 0; hh < GRP; ++hh) {
       if (!((mor >> hh) & 1u)) continue;   // no row of the unit kept by this head (warp-uniform)
-      float sc[8];
+      float sc[TPL];
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
+      for (int it = 0; it < TPL; ++it) {
         float d0 = 0.f;
 #pragma unroll
         for (int a = 0; a < DPL; ++a) d0 = fmaf(qv[hh][a], kf[it][a], d0);
@@ -744,7 +755,7 @@ __global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const Decod
       }
       float mb = sc[0];
 #pragma unroll
-      for (int it = 1; it < 8; ++it) mb = fmaxf(mb, sc[it]);
+      for (int it = 1; it < TPL; ++it) mb = fmaxf(mb, sc[it]);
       mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 16));
       const float mn = fmaxf(m[hh], mb);
       if (mn == -INFINITY) continue;   // nothing of this head in this warp yet (warp-uniform)
@@ -753,7 +764,7 @@ __global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const Decod
 #pragma unroll
       for (int a = 0; a < DPL; ++a) acc[hh][a] *= alpha;
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
+      for (int it = 0; it < TPL; ++it) {
         const float pe = ex2_approx(sc[it] - mn);   // -inf -> 0
         ls += pe;
 #pragma unroll
@@ -763,7 +774,7 @@ __global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const Decod
       m[hh] = mn;
     }
   }
-  // merge the two half-warps (same dims, same running max), then the 4 warps
+  // merge the two half-warps (same dims, same running max), then the NW warps
   float* red = reinterpret_cast<float*>(dsm + Lay::kRed);   // [warp][hh][D + 2]
 #pragma unroll
   for (int hh = 0; hh < GRP; ++hh) {
@@ -780,15 +791,15 @@ __global__ void __launch_bounds__(160, 1) cluster_stream_attn_kernel(const Decod
       r[D + 1] = l[hh];
     }
   }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
   if (!ok) return;
-  for (int x = threadIdx.x; x < GRP * D; x += 128) {
+  for (int x = threadIdx.x; x < GRP * D; x += NW * 32) {
     const int hh = x / D, c = x % D;
     float M = -INFINITY;
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, red[((size_t)w * kMaxGrp + hh) * (D + 2) + D]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, red[((size_t)w * kMaxGrp + hh) * (D + 2) + D]);
     float a = 0.f, L = 0.f;
     if (M != -INFINITY) {
-      for (int w = 0; w < 4; ++w) {
+      for (int w = 0; w < NW; ++w) {
         const float* r = red + ((size_t)w * kMaxGrp + hh) * (D + 2);
         if (r[D] == -INFINITY) continue;
         const float wgt = ex2_approx(r[D] - M);

@@ -173,9 +173,9 @@ def test_cluster_pack_kv_is_the_cluster_order_gather():
                                                       (1, 8, 1, 3072, 128, 2944, 48, 48)])
 def test_packed_cluster_decode_equals_gathered(B, Hq, Hkv, S, d, n_ctx, C, keep):
     """The cluster-ordered copy holds the same rows in the same order as the
-    token gather, and both kernels give each lane the same rows when a KV head
-    has at most 4 q-heads: the outputs are then identical bit for bit (with 8
-    the gather kernel takes 4 rows per lane and sums in another order)."""
+    token gather: the same clusters are kept, and the outputs differ only by
+    the fp32 summation order of the two kernels (each is checked against the
+    oracle in test_cluster_decode_matches_oracle)."""
     w = synth.make_decode("decode-b16-128k", device=DEV, B=B, S=S, Hq=Hq, Hkv=Hkv, d=d, seed=C + keep + 1)
     cent, _, off, tok = dsa.kmeans_clusters(w.k_cache, n_ctx, C, iters=2)
     packed = dsa.cluster_pack_kv(w.k_cache, w.v_cache, tok, n_ctx)
@@ -185,10 +185,8 @@ def test_packed_cluster_decode_equals_gathered(B, Hq, Hkv, S, d, n_ctx, C, keep)
     torch.cuda.synchronize()
     assert dsa.get_status() == 0
     assert torch.equal(si1, si2) and torch.equal(sc1, sc2)
-    if Hq // Hkv <= 4:
-        assert torch.equal(o1, o2)
-    else:
-        assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
+    err = (o1.float() - o2.float()).abs()
+    assert err.max().item() <= 1e-2 and err.mean().item() <= 1e-3
 
 
 def test_cluster_abi_rejects_bad_arguments():
