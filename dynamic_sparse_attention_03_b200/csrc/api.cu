@@ -183,7 +183,7 @@ int launch_decode(const DecodeParams& p, int B, int Hkv, int nchmax, size_t sel_
   decode_select_kernel<D, G, 256><<<B * Hkv, 256, sel_smem, st>>>(p);
   if ((rc = launch_check())) return rc;
   if ((rc = set_smem(decode_attn_kernel<D, G>, DecLayout<D>::kBytes))) return rc;
-  decode_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 160, DecLayout<D>::kBytes, st>>>(p);
+  decode_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), kDecThreads, DecLayout<D>::kBytes, st>>>(p);
   return launch_check();
 }
 

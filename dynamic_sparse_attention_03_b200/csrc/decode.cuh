@@ -31,6 +31,8 @@ namespace dsa {
 constexpr int kDecChunk = 64;      // union blocks per attention CTA
 constexpr int kDecStages = 4;
 constexpr int kMaxGrp = 8;         // q-heads per KV head supported by the decode path
+constexpr int kDecWarps = 8;       // consumer warps of decode_attn_kernel: 8 keys of each block per warp
+constexpr int kDecThreads = (kDecWarps + 1) * 32;   // plus the producer warp
 
 struct DecodeParams {
   const __nv_bfloat16* q;      // [B][Hq][D]
@@ -161,14 +163,15 @@ struct DecLayout {
   static constexpr int kStage = 2 * kBlkBytes;
   static constexpr int kRing = kDecStages * kStage;
   static constexpr int kRed = kRing;                            // warp partials
-  static constexpr int kRedBytes = 4 * kMaxGrp * (D + 2) * 4;
+  static constexpr int kRedBytes = kDecWarps * kMaxGrp * (D + 2) * 4;
   static constexpr int kBar = kRed + kRedBytes;
   static constexpr int kBytes = kBar + 2 * kDecStages * 8 + 16;
 };
 
 template <int D, int GRP>
-__global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(const DecodeParams p) {
   using Lay = DecLayout<D>;
+  constexpr int NW = kDecWarps, TPL = 32 / NW;   // keys per lane per block
   extern __shared__ __align__(16) uint8_t dsm[];
   const uint32_t sb = smem_u32(dsm);
   const int bg = blockIdx.x, chunk = blockIdx.y;
@@ -187,7 +190,7 @@ __global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), 4);
+      mbar_init(empty(s), NW);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -198,7 +201,7 @@ __global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams 
   const uint8_t* um = p.umask + (size_t)bg * p.nb + u0;
   const size_t head_base = (size_t)bg * p.S * D;
 
-  if (warp == 4) {
+  if (warp == NW) {
     // producer: one thread streams whole K and V blocks
     if (lane == 0) {
       int u = 0;
@@ -215,8 +218,8 @@ __global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams 
     }
     return;
   }
-  // consumers: warp w takes keys 16w .. 16w+15 of every block; the two half
-  // warps take alternate keys, lane%16 owns dims [8*(lane%16), +8).
+  // consumers: warp w takes keys 2 TPL w .. of every block; the two half
+  // warps take alternate keys, lane%16 owns dims [DPL*(lane%16), +DPL).
   constexpr int DPL = D / 16;            // dims per lane (8 at d=128, 4 at d=64)
   const int half = lane >> 4, dl = lane & 15;
   float qv[GRP][DPL];
@@ -240,11 +243,11 @@ __global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams 
     const uint8_t msk = um[u];
     const uint8_t* kb = dsm + s * Lay::kStage;
     const uint8_t* vb = kb + Lay::kBlkBytes;
-    // 8 keys per lane: key = 16*warp + 2*it + half
-    float kf[8][DPL], vf[8][DPL];
+    // TPL keys per lane: key = 2 TPL warp + 2 it + half
+    float kf[TPL][DPL], vf[TPL][DPL];
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int key = 16 * warp + 2 * it + half;
+    for (int it = 0; it < TPL; ++it) {
+      const int key = 2 * TPL * warp + 2 * it + half;
       if (DPL == 8) {
         const uint4 kr = *reinterpret_cast<const uint4*>(kb + key * D * 2 + dl * 16);
         const uint4 vr = *reinterpret_cast<const uint4*>(vb + key * D * 2 + dl * 16);
@@ -277,9 +280,9 @@ __global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams 
 #pragma unroll
     for (int hh = 0; hh < grp; ++hh) {
       if (!((msk >> hh) & 1u)) continue;   // block not kept by this head (warp-uniform)
-      float sc[8];
+      float sc[TPL];
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
+      for (int it = 0; it < TPL; ++it) {
         float d0 = 0.f;
 #pragma unroll
         for (int a = 0; a < DPL; ++a) d0 = fmaf(qv[hh][a], kf[it][a], d0);
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams 
       }
       float mb = sc[0];
 #pragma unroll
-      for (int it = 1; it < 8; ++it) mb = fmaxf(mb, sc[it]);
+      for (int it = 1; it < TPL; ++it) mb = fmaxf(mb, sc[it]);
       mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 16));
       const float mn = fmaxf(m[hh], mb);
       const float alpha = ex2_approx(m[hh] - mn);   // m = -inf -> 0
@@ -297,7 +300,7 @@ __global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams 
 #pragma unroll
       for (int a = 0; a < DPL; ++a) acc[hh][a] *= alpha;
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
+      for (int it = 0; it < TPL; ++it) {
         const float pe = ex2_approx(sc[it] - mn);
         ls += pe;
 #pragma unroll
@@ -307,7 +310,7 @@ __global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams 
       m[hh] = mn;
     }
   }
-  // merge the two half-warps (same dims, same running max), then the 4 warps
+  // merge the two half-warps (same dims, same running max), then the NW warps
   float* red = reinterpret_cast<float*>(dsm + Lay::kRed);   // [warp][hh][D + 2]
 #pragma unroll
   for (int hh = 0; hh < grp; ++hh) {
@@ -324,15 +327,15 @@ __global__ void __launch_bounds__(160, 1) decode_attn_kernel(const DecodeParams 
       r[D + 1] = l[hh];
     }
   }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
   if (!ok) return;
-  for (int x = threadIdx.x; x < grp * D; x += 128) {
+  for (int x = threadIdx.x; x < grp * D; x += NW * 32) {
     const int hh = x / D, c = x % D;
     float M = -INFINITY;
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, red[((size_t)w * kMaxGrp + hh) * (D + 2) + D]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, red[((size_t)w * kMaxGrp + hh) * (D + 2) + D]);
     float a = 0.f, L = 0.f;
     if (M != -INFINITY) {
-      for (int w = 0; w < 4; ++w) {
+      for (int w = 0; w < NW; ++w) {
         const float* r = red + ((size_t)w * kMaxGrp + hh) * (D + 2);
         const float wgt = ex2_approx(r[D] - M);
         a += wgt * r[c];

@@ -63,7 +63,7 @@ int launch(const DecodeParams& p, int B, int Hkv, int nchmax, size_t sel_smem, c
   if (cudaFuncSetAttribute(decode_attn_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DecLayout<D>::kBytes) != cudaSuccess)
     return DSA_ERR_CUDA;
-  decode_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), 160, DecLayout<D>::kBytes, st>>>(p);
+  decode_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), kDecThreads, DecLayout<D>::kBytes, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   decode_combine_kernel<D><<<B * (Hkv * G), 128, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
