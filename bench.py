@@ -329,7 +329,7 @@ def run_decode(args, local):
     import dynamic_sparse_attention_03_b200 as dsa
 
     dev = torch.device("cuda", local)
-    dw = synth.make_decode("decode-b16-128k", device=dev)
+    dw = synth.make_decode("decode-b16-128k", device=dev, B=args.decode_batch)
     p = dw.params
     cent = dsa.pool_keys(dw.k_cache)
     ws = dsa.Workspace(dev)
@@ -375,7 +375,7 @@ def run_decode(args, local):
     cent_ms = c0.elapsed_time(c1)
     cent_gbs = (B * Hkv * S * dd * 2 + bytes_cent) / (cent_ms * 1e-3) / 1e9
     del dw
-    return {"workload": "decode-b16-128k", "ms": round(ms, 4), "GB/s": round(gbs, 1),
+    return {"workload": f"decode-b{B}-128k", "ms": round(ms, 4), "GB/s": round(gbs, 1),
             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": total,
             "union_kv_blocks": union_blocks, "centroid_build_ms": round(cent_ms, 4),
             "centroid_build_GB/s": round(cent_gbs, 1), "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": src}
@@ -393,7 +393,7 @@ def run_cluster_decode(args, local):
     import dynamic_sparse_attention_03_b200 as dsa
 
     dev = torch.device("cuda", local)
-    dw = synth.make_decode("decode-b16-128k", device=dev)
+    dw = synth.make_decode("decode-b16-128k", device=dev, B=args.decode_batch)
     p = dw.params
     B, Hq, dd = dw.q.shape
     Hkv, S = dw.k_cache.shape[1], dw.k_cache.shape[2]
@@ -449,7 +449,7 @@ def run_cluster_decode(args, local):
     peaks, src = load_peaks()
     gbs = total / (ms * 1e-3) / 1e9
     del dw, packed
-    return {"workload": "decode-b16-128k, 2048 K-means clusters of the first S-64 keys, keep 512 + tail",
+    return {"workload": f"decode-b{B}-128k, {C} K-means clusters of the first S-64 keys, keep {keep} + tail",
             "ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
             "bytes_per_step": total, "union_tokens": union_tokens, "kv_layout": "cluster-ordered copy",
             "ms_token_gather": round(ms_gather, 4), "kmeans_build_ms": round(build_ms, 2),
@@ -620,6 +620,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--decode-batch", type=int, default=16,
+                    help="batch of the decode workloads (16 is the reported configuration; smaller for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
