@@ -167,6 +167,16 @@ def barrier(world: int):
 
 # ------------------------------------------------------------------ our arm
 
+def workload_config(workload: str, world: int) -> dict:
+    """The prefill workload's description, the same on both arms."""
+    p = synth.CONFIGS[workload]
+    kf, rho = p.get("k_fixed", 0), p.get("keep_ratio", 0.0)
+    return {"workload": workload, "Hq": p["Hq"], "Hkv": p["Hkv"], "seq_len": p["n"], "head_dim": p["d"],
+            "keep": f"k_fixed={kf}" if kf else f"ratio={rho}+sink+diag", "block": 64,
+            "l2": "inputs larger than L2 (Q 1.07 GB, K/V 268 MB each at 128K), no flush",
+            "parallelism": f"independent layer per GPU x{world}"}
+
+
 def run_ours(args, rank, world, local):
     import dynamic_sparse_attention_03_b200 as dsa
 
@@ -277,11 +287,7 @@ def run_ours(args, rank, world, local):
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "Hq": Hq, "Hkv": w.k.shape[0], "seq_len": n, "head_dim": d,
-                   "keep": f"k_fixed={kf}" if kf else f"ratio={rho}+sink+diag", "block": 64,
-                   "selected_block_density": round(density, 5),
-                   "l2": "inputs larger than L2 (Q 1.07 GB, K/V 268 MB each at 128K), no flush",
-                   "parallelism": f"independent layer per GPU x{world}"},
+        "config": dict(workload_config(args.workload, world), selected_block_density=round(density, 5)),
         "breakdown_ms": {"index": round(index_ms, 4), "attention": round(attn_ms, 4)},
         "index_roofline": index_roof,
         "index_reuse": reuse,
@@ -602,7 +608,7 @@ def run_reference(args, rank, world):
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": args.workload},
+            "config": workload_config(args.workload, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
