@@ -646,7 +646,7 @@ int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache,
   if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(centroids)) return DSA_ERR_INVALID_ARG;
   if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
   if (sel_idx && kcap < std::min(keep, C)) return DSA_ERR_CAPACITY;
-  const size_t sel_smem = (size_t)grp * C * 4 + (size_t)C * 12 + C;
+  const size_t sel_smem = (size_t)grp * C * 4 + (size_t)C * 12 + (size_t)(C + 1) * 4 + C;
   if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
   const int nchmax = (S + kClChunk - 1) / kClChunk;
   WsCarve c(ws);

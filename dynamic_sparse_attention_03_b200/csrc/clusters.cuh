@@ -331,8 +331,13 @@ __global__ void __launch_bounds__(NT) cluster_select_kernel(const ClusterParams 
   int32_t* cand = reinterpret_cast<int32_t*>(sc + (size_t)GRP * C);  // [C] non-empty cluster ids
   int32_t* tmp = cand + C;                                           // [C]
   int32_t* ubase = tmp + C;                                          // [C] union token offsets
-  uint8_t* mask = reinterpret_cast<uint8_t*>(ubase + C);             // [C]
-  const int32_t* off = cp.off + (size_t)bg * (C + 1);
+  int32_t* off = ubase + C;                                          // [C + 1] the cluster -> key offsets
+  uint8_t* mask = reinterpret_cast<uint8_t*>(off + C + 1);           // [C]
+  // the offsets come in once, coalesced: the union loop below reads them per
+  // cluster, which from global memory was a chain of dependent loads per warp
+  const int32_t* goff = cp.off + (size_t)bg * (C + 1);
+  for (int x = threadIdx.x; x <= C; x += NT) off[x] = goff[x];
+  __syncthreads();
   // non-empty clusters, ascending (block scan over per-thread ranges)
   const int per = (C + NT - 1) / NT;
   const int c0 = min(C, (int)threadIdx.x * per), c1 = min(C, c0 + per);
