@@ -19,8 +19,9 @@
 //           chunks are read whole and the window is their range;
 //   pass 1 (approximate): a 256-bin histogram of the row in that window gives
 //           the bin holding the row's e-th largest score;
-//   pass 2 (exact: Q̄hi·K̄hi + Q̄hi·K̄lo + Q̄lo·K̄hi): scores above that bin (widened by a quarter bin on
-//           each side) are kept at once, as bits of a per-chunk mask in
+//   pass 2 (exact: Q̄hi·K̄hi + Q̄hi·K̄lo + Q̄lo·K̄hi): scores above that bin
+//           (widened by a quarter bin on each side) are kept at once, as bits
+//           of a per-chunk mask in
 //           scratch memory; scores inside it are buffered as (key, id)
 //           candidates.  If the kept count and the candidates bracket e, the
 //           e-th largest key T and the number of T-valued ids to keep are
@@ -35,7 +36,7 @@
 // same scores bit for bit (the same MMA sequence), so the passes agree.
 //
 // A second kernel writes the lists from the masks, one warp per query block
-// (ascending ids, coalesced stores).
+// (ascending ids; each lane writes the ids of one mask word).
 #pragma once
 
 #include <cuda_bf16.h>
