@@ -75,6 +75,25 @@ def test_block_index_and_attention(n, d, Hq, Hkv, rho):
     check_attention(o, ref, f"n={n} d={d}")
 
 
+@pytest.mark.parametrize("q_scale,k_scale", [(2.0 ** 12, 2.0 ** -12), (1000.0, 0.001), (0.003, 0.02), (37.0, 1.0)])
+def test_block_index_input_scales(q_scale, k_scale):
+    """The index operands are FP16 splits of the pooled means after a power-of-
+    two scale per query block and per KV head, so the index must not depend on
+    the inputs' magnitude: large and small Q and K give the oracle's sets, and
+    power-of-two scales give exactly the unscaled lists."""
+    n, d, Hq, Hkv, rho = 4096, 128, 8, 2, 0.10
+    w = synth.make_prefill("llama3-8b-32k-bs10", device=DEV, n=n, Hq=Hq, Hkv=Hkv, d=d, seed=77)
+    qs = (w.q.float() * q_scale).to(torch.bfloat16)
+    ks = (w.k.float() * k_scale).to(torch.bfloat16)
+    bi, bc = dsa.sparse_index_estimate(qs, ks, keep_ratio=rho)
+    got = lists_from_gpu(bi, bc)
+    _, info, _ = oracle.block_index(f64(qs), f64(ks), keep_ratio=rho)
+    check_block_index(got, info, f"scales {q_scale}, {k_scale}")
+    if math.log2(q_scale).is_integer() and math.log2(k_scale).is_integer():
+        bi0, bc0 = dsa.sparse_index_estimate(w.q, w.k, keep_ratio=rho)
+        assert torch.equal(bi, bi0) and torch.equal(bc, bc0)
+
+
 def _random_lists(rng, Hq, nqb, kcap, p_keep, with_cols, ccap=0, empty_rows=()):
     bi = -np.ones((Hq, nqb, kcap), np.int32)
     bc = np.zeros((Hq, nqb), np.int32)
