@@ -94,6 +94,30 @@ def test_block_index_input_scales(q_scale, k_scale):
         assert torch.equal(bi, bi0) and torch.equal(bc, bc0)
 
 
+def test_block_index_exact_ties_take_the_lower_blocks():
+    """Key blocks drawn from four repeated vectors: every row's scores take a
+    few values, each shared by many blocks, so the e-th largest sits inside a
+    large group of exactly equal scores (equal in fp32 on the GPU and in fp64
+    in the oracle).  The selection's window then holds more candidates than
+    its buffer and the exact fallback passes run (value histogram, radix
+    passes on the keys, threshold sweep); the ties must go to the lower
+    blocks, so every row matches the oracle exactly."""
+    n, d, Hq, Hkv, rho = 32768, 128, 4, 1, 0.10
+    w = synth.make_prefill("llama3-8b-32k-bs10", device=DEV, n=n, Hq=Hq, Hkv=Hkv, d=d, seed=5)
+    nqb = n // 64
+    g = torch.Generator(device="cpu").manual_seed(123)
+    types = torch.randn((4, d), generator=g).to(torch.bfloat16)
+    pick = torch.randint(0, 4, (nqb,), generator=g)
+    k = types[pick].repeat_interleave(64, dim=0).reshape(1, n, d).contiguous().to(DEV)
+    bi, bc = dsa.sparse_index_estimate(w.q, k, keep_ratio=rho)
+    torch.cuda.synchronize()
+    assert dsa.get_status() == 0
+    got = lists_from_gpu(bi, bc)
+    _, info, _ = oracle.block_index(f64(w.q), f64(k), keep_ratio=rho)
+    stats = check_block_index(got, info, "exact ties")
+    assert stats.get("ambiguous", 0) == 0, stats
+
+
 def _random_lists(rng, Hq, nqb, kcap, p_keep, with_cols, ccap=0, empty_rows=()):
     bi = -np.ones((Hq, nqb, kcap), np.int32)
     bc = np.zeros((Hq, nqb), np.int32)
