@@ -137,6 +137,12 @@ def _need_dtype(t, dt, name):
         raise TypeError(f"{name} must be {dt}, got {t.dtype}")
 
 
+def _need_shape(t, shape, name):
+    # the C entry points trust the sizes they are given: check them here
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
 class Workspace:
     """Device scratch for the library calls, grown on demand, one per device.
 
@@ -383,12 +389,19 @@ def cluster_pack_kv(k_cache: torch.Tensor, v_cache: torch.Tensor, tokens: torch.
     _need_cuda(k_cache, v_cache, tokens)
     _need_dtype(k_cache, torch.bfloat16, "k_cache")
     _need_dtype(v_cache, torch.bfloat16, "v_cache")
+    _need_dtype(tokens, torch.int32, "tokens")
     B, Hkv, S, d = k_cache.shape
+    _need_shape(v_cache, k_cache.shape, "v_cache")
+    _need_shape(tokens, (B, Hkv, int(n_ctx)), "tokens")
     if out is None:
         kp = torch.empty((B, Hkv, int(n_ctx), d), dtype=torch.bfloat16, device=k_cache.device)
         vp = torch.empty_like(kp)
     else:
         kp, vp = out
+        _need_cuda(kp, vp)
+        for t, nm in ((kp, "k_packed"), (vp, "v_packed")):
+            _need_dtype(t, torch.bfloat16, nm)
+            _need_shape(t, (B, Hkv, int(n_ctx), d), nm)
     _check(load_library().cluster_pack_kv(_ptr(k_cache), _ptr(v_cache), _ptr(tokens), B, Hkv, S, d, int(n_ctx),
                                           _ptr(kp), _ptr(vp), _stream(k_cache.device)), "cluster_pack_kv")
     return kp, vp
@@ -409,9 +422,20 @@ def cluster_decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.T
     kp, vp = packed if packed is not None else (None, None)
     _need_cuda(q, k_cache, v_cache, centroids, offsets, tokens, out, kp, vp)
     _need_dtype(centroids, torch.float32, "centroids")
+    _need_dtype(offsets, torch.int32, "offsets")
+    _need_dtype(tokens, torch.int32, "tokens")
     B, Hq, d = q.shape
     Hkv, S = k_cache.shape[1], k_cache.shape[2]
     C = centroids.shape[2]
+    _need_shape(k_cache, (B, Hkv, S, d), "k_cache")
+    _need_shape(v_cache, (B, Hkv, S, d), "v_cache")
+    _need_shape(centroids, (B, Hkv, C, d), "centroids")
+    _need_shape(offsets, (B, Hkv, C + 1), "offsets")
+    _need_shape(tokens, (B, Hkv, int(n_ctx)), "tokens")
+    if kp is not None:
+        for t, nm in ((kp, "k_packed"), (vp, "v_packed")):
+            _need_dtype(t, torch.bfloat16, nm)
+            _need_shape(t, (B, Hkv, int(n_ctx), d), nm)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     kcap = max(min(int(keep), C), 1)

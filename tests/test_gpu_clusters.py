@@ -197,6 +197,8 @@ def test_cluster_abi_rejects_bad_arguments():
         dsa.kmeans_clusters(kc, 300, 8, iters=1)        # context past the cache
     with pytest.raises(dsa.DSAError):
         dsa.kmeans_clusters(kc, 256, 8, iters=0)
-    tok = torch.zeros((1, 1, 256), dtype=torch.int32, device=DEV)
+    tok = torch.zeros((1, 1, 300), dtype=torch.int32, device=DEV)
     with pytest.raises(dsa.DSAError):
-        dsa.cluster_pack_kv(kc, kc, tok, 300)          # context past the cache
+        dsa.cluster_pack_kv(kc, kc, tok, 300)          # context past the cache (the library's check)
+    with pytest.raises(ValueError):
+        dsa.cluster_pack_kv(kc, kc, tok[..., :200], 256)   # tokens of the wrong length (the binding's check)
