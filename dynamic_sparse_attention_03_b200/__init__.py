@@ -213,11 +213,18 @@ def sparse_index_estimate(q: torch.Tensor, k: torch.Tensor, k_fixed: int = 0, ke
         raise ValueError("k must be [Hkv][n][d] with q's n and d")
     nqb = n // 64
     if kcap is None:
-        kcap = block_index_capacity(n, k_fixed, keep_ratio)
+        kcap = block_idx.shape[-1] if block_idx is not None else block_index_capacity(n, k_fixed, keep_ratio)
     if block_idx is None:
         block_idx = torch.empty((Hq, nqb, kcap), dtype=torch.int32, device=q.device)
     if block_cnt is None:
         block_cnt = torch.empty((Hq, nqb), dtype=torch.int32, device=q.device)
+    _need_dtype(block_idx, torch.int32, "block_idx")
+    _need_dtype(block_cnt, torch.int32, "block_cnt")
+    _need_shape(block_idx, (Hq, nqb, kcap), "block_idx")
+    _need_shape(block_cnt, (Hq, nqb), "block_cnt")
+    if pooled_k is not None:
+        _need_dtype(pooled_k, torch.float32, "pooled_k")
+        _need_shape(pooled_k, (Hkv, nqb, d), "pooled_k")
     args = [_ptr(q), _ptr(k), Hq, Hkv, n, d, 64, int(k_fixed), float(keep_ratio), _ptr(block_idx),
             _ptr(block_cnt), int(kcap), _ptr(pooled_k)]
     _call_with_ws("sparse_index_estimate", args, q.device, ws)
@@ -233,6 +240,8 @@ def pool_keys(k: torch.Tensor, out: Optional[torch.Tensor] = None, ws: Optional[
     rows = int(math.prod(lead)) if lead else 1
     if out is None:
         out = torch.empty(lead + (S // 64, d), dtype=torch.float32, device=k.device)
+    _need_dtype(out, torch.float32, "out")
+    _need_shape(out, lead + (S // 64, d), "out")
     args = [None, _ptr(k), 0, rows, S, d, 64, 0, 0.0, None, None, 0, _ptr(out)]
     _call_with_ws("sparse_index_estimate", args, k.device, ws)
     return out
@@ -250,6 +259,7 @@ def vertical_slash_index(q: torch.Tensor, k: torch.Tensor, n_vert: int, n_slash:
     _need_dtype(k, torch.bfloat16, "k")
     Hq, n, d = q.shape
     Hkv = k.shape[0]
+    _need_shape(k, (Hkv, n, d), "k")
     nqb = n // 64
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dev = q.device
@@ -267,6 +277,10 @@ def vertical_slash_index(q: torch.Tensor, k: torch.Tensor, n_vert: int, n_slash:
         col_idx=torch.empty((Hq, nqb, ccap), dtype=torch.int32, device=dev),
         col_cnt=torch.empty((Hq, nqb), dtype=torch.int32, device=dev),
     )
+    for nm, shape in (("vert_idx", (Hq, n_vert)), ("slash_off", (Hq, n_slash)), ("block_idx", (Hq, nqb, kcap)),
+                      ("block_cnt", (Hq, nqb)), ("col_idx", (Hq, nqb, ccap)), ("col_cnt", (Hq, nqb))):
+        _need_dtype(out[nm], torch.int32, nm)
+        _need_shape(out[nm], shape, nm)
     args = [_ptr(q), _ptr(k), Hq, Hkv, n, d, int(last_q), int(n_vert), int(n_slash), float(scale),
             _ptr(out["vert_idx"]), _ptr(out["slash_off"]), _ptr(out["block_idx"]), _ptr(out["block_cnt"]), kcap,
             _ptr(out["col_idx"]), _ptr(out["col_cnt"]), ccap]
@@ -286,15 +300,44 @@ def block_sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blo
         _need_dtype(t, torch.bfloat16, nm)
     Hq, n, d = q.shape
     Hkv = k.shape[0]
+    nqb = n // 64
+    _need_shape(k, (Hkv, n, d), "k")
+    _need_shape(v, (Hkv, n, d), "v")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
+    _need_dtype(o, torch.bfloat16, "out")
+    _need_shape(o, (Hq, n, d), "out")
     lse = torch.empty((Hq, n), dtype=torch.float32, device=q.device) if return_lse else None
     kcap = block_idx.shape[-1]
     ccap = col_idx.shape[-1] if col_idx is not None else 0
+    _need_dtype(block_idx, torch.int32, "block_idx")
+    _need_dtype(block_cnt, torch.int32, "block_cnt")
+    _need_shape(block_idx, (Hq, nqb, kcap), "block_idx")
+    _need_shape(block_cnt, (Hq, nqb), "block_cnt")
+    if (col_idx is None) != (col_cnt is None):
+        raise ValueError("col_idx and col_cnt go together")
+    if col_idx is not None:
+        _need_dtype(col_idx, torch.int32, "col_idx")
+        _need_dtype(col_cnt, torch.int32, "col_cnt")
+        _need_shape(col_idx, (Hq, nqb, ccap), "col_idx")
+        _need_shape(col_cnt, (Hq, nqb), "col_cnt")
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(o), Hq, Hkv, n, d, float(scale), _ptr(block_idx), _ptr(block_cnt), kcap,
             _ptr(col_idx), _ptr(col_cnt), ccap, _ptr(lse)]
     _call_with_ws("block_sparse_attn_fwd", args, q.device, ws)
     return (o, lse) if return_lse else o
+
+
+def _check_decode_inputs(q, k_cache, v_cache, centroids, out):
+    B, Hq, d = q.shape
+    Hkv, S = k_cache.shape[1], k_cache.shape[2]
+    for t, nm in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need_dtype(t, torch.bfloat16, nm)
+    _need_shape(k_cache, (B, Hkv, S, d), "k_cache")
+    _need_shape(v_cache, (B, Hkv, S, d), "v_cache")
+    _need_shape(centroids, (B, Hkv, S // 64, d), "centroids")
+    if out is not None:
+        _need_dtype(out, torch.bfloat16, "out")
+        _need_shape(out, (B, Hq, d), "out")
 
 
 def sparse_decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, centroids: torch.Tensor,
@@ -306,6 +349,7 @@ def sparse_decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Te
     _need_dtype(centroids, torch.float32, "centroids")
     B, Hq, d = q.shape
     Hkv, S = k_cache.shape[1], k_cache.shape[2]
+    _check_decode_inputs(q, k_cache, v_cache, centroids, out)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     nb = S // 64
@@ -330,6 +374,7 @@ def sparse_decode_attn_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
     _need_dtype(centroids, torch.float32, "centroids")
     B, Hq, d = q.shape
     Hkv, S = k_cache.shape[1], k_cache.shape[2]
+    _check_decode_inputs(q, k_cache, v_cache, centroids, out)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     nb = S // 64
