@@ -3,8 +3,9 @@ split into hi + lo after a power-of-two scale (per query block for Q̄, per KV
 head for K̄).  This checks, in NumPy, the precision that choice gives: the
 split carries about 22 bits, the three-product score is within 2^-19 of
 |q||k| of the exact dot product (2^-23 on these draws: far inside the 1e-4
-near-tie rule), and a single hi*hi product is not (2^-13 on these draws).  It restates the arithmetic of
-the split, not the kernels, and imports neither the library nor the oracle."""
+near-tie rule), and a single hi*hi product is not (2^-13 on these draws).
+It restates the arithmetic of the split, not the kernels, and imports neither
+the library nor the oracle."""
 
 import numpy as np
 
