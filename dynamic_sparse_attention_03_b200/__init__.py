@@ -171,15 +171,30 @@ def _workspace(dev: torch.device, ws: Optional[Workspace]) -> Workspace:
     return _ws_cache[key]
 
 
+def _on_device(dev):
+    """Context that makes dev the current CUDA device for a library call."""
+    return torch.cuda.device(dev)
+
+
+def _dev_index(dev) -> int:
+    dev = torch.device(dev)
+    return dev.index if dev.index is not None else torch.cuda.current_device()
+
+
 def _call_with_ws(name, args_before_ws, dev, ws):
-    """Query the workspace size (ws = NULL), then call with the buffer."""
+    """Query the workspace size (ws = NULL), then call with the buffer.  The
+    tensors' device is made current for the call: the library sizes grids and
+    sets kernel attributes for the current device."""
     lib = load_library()
     fn = getattr(lib, name)
     size = ctypes.c_size_t(0)
-    _check(fn(*args_before_ws, None, ctypes.byref(size), _stream(dev)), name)
-    w = _workspace(dev, ws)
-    buf = w.ensure(size.value)
-    _check(fn(*args_before_ws, _ptr(buf), ctypes.byref(size), _stream(dev)), name)
+    with _on_device(dev):
+        _check(fn(*args_before_ws, None, ctypes.byref(size), _stream(dev)), name)
+        w = _workspace(dev, ws)
+        if _dev_index(w.device) != _dev_index(dev):
+            raise ValueError(f"workspace is on {w.device}, tensors on {dev}")
+        buf = w.ensure(size.value)
+        _check(fn(*args_before_ws, _ptr(buf), ctypes.byref(size), _stream(dev)), name)
     return w
 
 
@@ -187,7 +202,8 @@ def get_status(ws: Optional[Workspace] = None, device=None) -> int:
     """Synchronize the current stream and return (and clear) the device status word."""
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     w = _workspace(dev, ws)
-    return load_library().dsa_get_status(_ptr(w.buf), _stream(dev))
+    with _on_device(w.device):
+        return load_library().dsa_get_status(_ptr(w.buf), _stream(w.device))
 
 
 def block_index_capacity(n: int, k_fixed: int = 0, keep_ratio: float = 0.0) -> int:
@@ -383,9 +399,11 @@ def sparse_decode_attn_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
     if return_sel:
         sel_idx = torch.empty((B, Hq, kcap), dtype=torch.int32, device=q.device)
         sel_cnt = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
-    rc = load_library().sparse_decode_attn_static(
-        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(centroids), B, Hq, Hkv, S, d, int(keep), int(force_last),
-        float(scale), _ptr(o), _ptr(sel_idx), _ptr(sel_cnt), kcap, _stream(q.device))
+    # the library's scratch array of the current device is used: make q's current
+    with _on_device(q.device):
+        rc = load_library().sparse_decode_attn_static(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(centroids), B, Hq, Hkv, S, d, int(keep), int(force_last),
+            float(scale), _ptr(o), _ptr(sel_idx), _ptr(sel_cnt), kcap, _stream(q.device))
     _check(rc, "sparse_decode_attn_static")
     return (o, sel_idx, sel_cnt) if return_sel else o
 
@@ -398,8 +416,9 @@ def a_shape_index(Hq: int, n: int, n_sink: int, n_local: int, device=None):
     kcap = max(1, min(nqb, n_sink + n_local))
     bi = torch.empty((Hq, nqb, kcap), dtype=torch.int32, device=dev)
     bc = torch.empty((Hq, nqb), dtype=torch.int32, device=dev)
-    _check(load_library().a_shape_index(Hq, n, n_sink, n_local, _ptr(bi), _ptr(bc), kcap, _stream(dev)),
-           "a_shape_index")
+    with _on_device(dev):
+        _check(load_library().a_shape_index(Hq, n, n_sink, n_local, _ptr(bi), _ptr(bc), kcap, _stream(dev)),
+               "a_shape_index")
     return bi, bc
 
 
@@ -447,8 +466,10 @@ def cluster_pack_kv(k_cache: torch.Tensor, v_cache: torch.Tensor, tokens: torch.
         for t, nm in ((kp, "k_packed"), (vp, "v_packed")):
             _need_dtype(t, torch.bfloat16, nm)
             _need_shape(t, (B, Hkv, int(n_ctx), d), nm)
-    _check(load_library().cluster_pack_kv(_ptr(k_cache), _ptr(v_cache), _ptr(tokens), B, Hkv, S, d, int(n_ctx),
-                                          _ptr(kp), _ptr(vp), _stream(k_cache.device)), "cluster_pack_kv")
+    with _on_device(k_cache.device):
+        _check(load_library().cluster_pack_kv(_ptr(k_cache), _ptr(v_cache), _ptr(tokens), B, Hkv, S, d,
+                                              int(n_ctx), _ptr(kp), _ptr(vp), _stream(k_cache.device)),
+               "cluster_pack_kv")
     return kp, vp
 
 

@@ -12,8 +12,11 @@
 // The scratch is one file-scope __device__ array of kStaticScratchBytes
 // (32 MiB); every GPU that loads the library keeps it until the process exits.
 // Host code must not use the array's name as a device address (on the host it
-// names a host-side shadow), so the device address is looked up once per
-// device with cudaGetSymbolAddress, with that device current, and cached.
+// names a host-side shadow), so the device address is looked up with
+// cudaGetSymbolAddress, with the device current, once per device and context:
+// a device reset makes a new primary context, in which the module is loaded
+// again and the array may move, so a context change triggers a new lookup.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -32,20 +35,54 @@ constexpr int kMaxDevices = 64;
 __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
 
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+struct ScratchAddr {
+  unsigned long long ctx_id;   // context the address belongs to (0: none yet)
+  void* ptr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up on the
-// first call per device).  nullptr if the lookup fails.
+// The current context's unique id (driver entry points, found once); 0 if unknown.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess && cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) ==
+        cudaSuccess && qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<GetCurrent>(a);
+      get_id = reinterpret_cast<GetId>(b);
+    }
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device, looked up on the
+// first call per device and again whenever the device's context has changed
+// (or its id cannot be read).  nullptr if the lookup fails.
 void* scratch_on_current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  const unsigned long long id = current_context_id();   // 0 before the context exists
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  ScratchAddr& e = g_scratch_addr[dev];
+  if (!e.ptr || id == 0 || e.ctx_id != id) {
     void* p = nullptr;
+    // (creates the device's primary context if there is none yet)
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
-    g_scratch_addr[dev] = p;
+    e.ptr = p;
+    e.ctx_id = current_context_id();
   }
-  return g_scratch_addr[dev];
+  return e.ptr;
 }
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }

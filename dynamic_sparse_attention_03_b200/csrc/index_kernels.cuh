@@ -31,8 +31,8 @@ constexpr int kBlock = 64;
 //
 //  out     (optional) the fp32 means;
 //  amax    (optional) atomic max of the block's max |mean| per group of
-//          rows_per_group blocks (float bits: non-negative floats order as
-//          unsigned integers);
+//          rows_per_group blocks, the group's first block excluded (float
+//          bits: non-negative floats order as unsigned integers);
 //  hi, lo  (optional) the split with the block's own scale (query blocks).
 // CTAs past the nblocks pooling ones convert conv_rows fp32 rows of conv_src
 // (8 per CTA) into conv_hi / conv_lo with the scale of their group's amax
@@ -120,7 +120,13 @@ __global__ void __launch_bounds__(256) pool_blocks_kernel(
   float bm = 0.f;
 #pragma unroll
   for (int w = 0; w < 8; ++w) bm = fmaxf(bm, wmax[w]);
-  if (amax && threadIdx.x == 0) atomicMax(amax + blk / rows_per_group, __float_as_uint(bm));
+  // The first block of each group (the forced sink block of a KV head) stays
+  // out of the group's max: sink keys are often far larger than the rest, and
+  // a scale set by them would push the other blocks' low halves toward the
+  // FP16 subnormal range.  The sink's own split may then overflow to inf; its
+  // score column is never ranked (it is always kept).
+  if (amax && threadIdx.x == 0 && blk % rows_per_group != 0)
+    atomicMax(amax + blk / rows_per_group, __float_as_uint(bm));
   if (hi && c < D) {
     __half h, l;
     split_f16(mean, pow2_scale_for(bm), h, l);

@@ -182,10 +182,14 @@ int sparse_decode_attn(const void* q, const void* k_cache, const void* v_cache, 
  *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *    Every GPU that loads the library holds the 32 MiB array until exit.
  *  - Sizes whose scratch exceeds 32 MiB are rejected with DSA_ERR_CAPACITY
- *    before any launch (e.g. B=16, Hq=32, Hkv=8, S=131072, d=128 needs ~9.9 MB).
+ *    before any launch.  The scratch is 256 B + B·Hkv·nb·5 B (union lists and
+ *    masks) + B·Hkv·4 B + B·Hq·nc·(d+2)·4 B (chunk partials, nc = ceil(nb/64))
+ *    + B·Hq·nb·4 B (block scores), nb = S/64, each part rounded up to 256 B:
+ *    B=16, Hq=32, Hkv=8, S=131072, d=128 needs 14.0 MB.
  *  - The first call on a device looks up the array's device address on that
  *    device (make the device current first); make that first call before any
- *    stream capture.
+ *    stream capture.  The address is kept per device context: after a device
+ *    reset (a new primary context) the next call looks it up again.
  *  - All calls share the one array, which keeps the previous call's contents;
  *    each call clears the status word it needs zeroed.  Calls that overlap on
  *    the GPU (different streams, or other host threads, without ordering

@@ -3,6 +3,8 @@
 library is replaced by a stub that records the calls, so nothing runs on a
 device."""
 
+import contextlib
+
 import pytest
 import torch
 
@@ -25,6 +27,7 @@ def calls(monkeypatch):
     monkeypatch.setattr(dsa, "_call_with_ws", lambda name, args, dev, ws: seen.append(name))
     monkeypatch.setattr(dsa, "load_library", lambda *a, **k: StubLib())
     monkeypatch.setattr(dsa, "_stream", lambda dev: None)
+    monkeypatch.setattr(dsa, "_on_device", lambda dev: contextlib.nullcontext())
     return seen
 
 

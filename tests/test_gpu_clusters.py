@@ -113,10 +113,13 @@ def test_kmeans_rounds_are_self_consistent():
 @pytest.mark.parametrize("packed", [False, True])
 @pytest.mark.parametrize("B,Hq,Hkv,S,d,n_ctx,C,keep", [(2, 8, 2, 4096, 128, 4032, 64, 16),
                                                       (1, 4, 4, 2048, 64, 2048, 32, 8),
-                                                      (1, 8, 1, 3072, 128, 2944, 48, 48)])
+                                                      (1, 8, 1, 3072, 128, 2944, 48, 48),
+                                                      (1, 4, 1, 16384, 128, 16320, 256, 192)])
 def test_cluster_decode_matches_oracle(B, Hq, Hkv, S, d, n_ctx, C, keep, packed):
     """Both forms of the decode: rows gathered by token id, and rows streamed
-    from the cluster-ordered copy."""
+    from the cluster-ordered copy.  The last case keeps about 12K rows of one
+    (batch, KV head), more than one 4096-row chunk of the kernel, so the
+    per-chunk partial softmax states are merged."""
     w = synth.make_decode("decode-b16-128k", device=DEV, B=B, S=S, Hq=Hq, Hkv=Hkv, d=d, seed=C + keep)
     cent, assign, off, tok = dsa.kmeans_clusters(w.k_cache, n_ctx, C, iters=2)
     pk = dsa.cluster_pack_kv(w.k_cache, w.v_cache, tok, n_ctx) if packed else None

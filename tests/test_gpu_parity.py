@@ -94,6 +94,30 @@ def test_block_index_input_scales(q_scale, k_scale):
         assert torch.equal(bi, bi0) and torch.equal(bc, bc0)
 
 
+@pytest.mark.parametrize("where,p", [("sink", 8), ("sink", 12), ("sink", 16), ("sink", 20), ("sink", 24),
+                                     ("candidate", 8), ("candidate", 12), ("candidate", 16), ("candidate", 20)])
+def test_block_index_outlier_key_block(where, p):
+    """One key block 2^p times larger than the rest, as attention-sink keys
+    often are.  The FP16 split of the pooled keys is scaled once per KV head,
+    so an outlier that set that scale would push every other block's low half
+    toward the subnormal range; the forced sink block is therefore left out of
+    the scale (its own score is never ranked).  The rows keep 30% of their
+    candidates, so the boundary falls inside the Gaussian bulk where scores
+    are close, and 512 query blocks make long rows."""
+    n, d, Hq, Hkv, rho = 32768, 128, 2, 1, 0.3
+    w = synth.make_prefill("llama3-8b-32k-bs10", device=DEV, n=n, Hq=Hq, Hkv=Hkv, d=d, seed=78)
+    blk = 0 if where == "sink" else 37
+    k = w.k.float()
+    k[:, blk * 64:(blk + 1) * 64] *= 2.0 ** p
+    k = k.to(torch.bfloat16).contiguous()
+    bi, bc = dsa.sparse_index_estimate(w.q, k, keep_ratio=rho)
+    torch.cuda.synchronize()
+    assert dsa.get_status() == 0
+    got = lists_from_gpu(bi, bc)
+    _, info, _ = oracle.block_index(f64(w.q), f64(k), keep_ratio=rho)
+    check_block_index(got, info, f"outlier {where} x2^{p}")
+
+
 def test_block_index_exact_ties_take_the_lower_blocks():
     """Key blocks drawn from four repeated vectors: every row's scores take a
     few values, each shared by many blocks, so the e-th largest sits inside a

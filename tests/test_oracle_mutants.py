@@ -12,6 +12,7 @@ import oracle
 from oracle import attention as oatt
 from oracle import blocksel as obi
 from oracle import decode as odec
+from oracle import ties as oties
 from oracle import vslash as ovs
 import tests.test_oracle_pins as pins
 
@@ -48,6 +49,69 @@ def _high_tie_select(scores, cand, e):
 def _slash_plus(q, k, last_q, scale, heads=None):
     vert, slash = ovs.__dict__["_orig_vs"](q, k, last_q, scale, heads)
     return vert, {h: np.roll(s, 1) for h, s in slash.items()}
+
+
+def _tie_dropping(branch):
+    """The near-tie comparison with one rejection branch removed: a set that
+    only that branch rejects is accepted instead."""
+    real = oties.__dict__["_orig_compare"]
+
+    def cmp(got, forced, cand, scores, e, rel=oties.REL):
+        st = real(got, forced, cand, scores, e, rel)
+        return "ambiguous" if st == "MISMATCH: " + branch else st
+    return cmp
+
+
+def _tie_lower_bound_variant(sign, use_abs):
+    """The near-tie comparison with the lower bound written as
+    t_(k+1) + sign * rel * (|t_(k+1)| if use_abs else t_(k+1))."""
+    def cmp(got, forced, cand, scores, e, rel=oties.REL):
+        got = np.asarray(got, dtype=np.int64)
+        forced = np.asarray(forced, dtype=np.int64)
+        if got.size and np.any(np.diff(got) <= 0):
+            return "MISMATCH: not strictly ascending"
+        if not np.all(np.isin(forced, got)):
+            return "MISMATCH: a forced element is missing"
+        chosen = np.setdiff1d(got, forced)
+        if chosen.size != e:
+            return "MISMATCH: count"
+        if not np.all(np.isin(chosen, cand)):
+            return "MISMATCH: an id outside the candidates"
+        if e == 0 or e == cand.size:
+            return "exact"
+        order = np.lexsort((cand, -scores))
+        if np.array_equal(np.sort(cand[order[:e]]), chosen):
+            return "exact"
+        tk, tk1 = scores[order[e - 1]], scores[order[e]]
+        if abs(tk - tk1) >= rel * max(abs(tk), abs(tk1)):
+            return "MISMATCH: no near tie"
+        upper = tk + rel * abs(tk)
+        lower = tk1 + sign * rel * (abs(tk1) if use_abs else tk1)
+        s_of = dict(zip(cand.tolist(), scores.tolist()))
+        if not np.all(np.isin(cand[scores > upper], chosen)):
+            return "MISMATCH: a clearly higher candidate was dropped"
+        if any(s_of[int(c)] < lower for c in chosen):
+            return "MISMATCH: a clearly lower candidate was kept"
+        return "ambiguous"
+    return cmp
+
+
+TIE_MUTANTS = {
+    "tie_no_lower_bound": lambda: _tie_dropping("a clearly lower candidate was kept"),
+    "tie_no_ascending": lambda: _tie_dropping("not strictly ascending"),
+    "tie_no_outside": lambda: _tie_dropping("an id outside the candidates"),
+    "tie_lower_bound_sign": lambda: _tie_lower_bound_variant(+1.0, True),
+    "tie_lower_bound_no_abs": lambda: _tie_lower_bound_variant(-1.0, False),
+}
+
+
+@pytest.mark.parametrize("case", sorted(TIE_MUTANTS))
+def test_planted_tie_rule_mistake_is_caught(case, monkeypatch):
+    monkeypatch.setitem(oties.__dict__, "_orig_compare", oties.compare_index_sets)
+    mutant = TIE_MUTANTS[case]()
+    monkeypatch.setattr(oracle, "compare_index_sets", mutant)
+    with pytest.raises(AssertionError):
+        pins.test_tie_rule_every_rejection_branch()
 
 
 @pytest.mark.parametrize("case", ["sum_pool", "transposed", "no_causal", "unscaled", "high_tie", "slash_shift"])

@@ -329,6 +329,45 @@ def test_tie_rule():
     assert oracle.compare_index_sets([1, 2, 4, 8], forced, cand, scores, 2).startswith("MISMATCH")
 
 
+def test_tie_rule_every_rejection_branch():
+    """Each way a set can break the near-tie rule, in a row that has a near tie
+    at the boundary (ids 4 and 3 score 3.0000001 and 3.0, 3 kept), so that only
+    the branch under test can reject it:
+
+    * a clearly lower candidate kept: {1, 2, 5} has the right count and both
+      clearly higher ids (5.0, 4.0), but id 5 scores 1.0, below the (k+1)-th
+      score 3.0 by far more than 1e-4 relative;
+    * a candidate just inside the lower bound is accepted (id 3, exactly the
+      (k+1)-th score), and one scoring 0.99995 of it is not;
+    * ids not strictly ascending, or repeated;
+    * an id that is not a candidate (9 > 8, the last forced id)."""
+    cand = np.arange(1, 8)
+    scores = np.array([5.0, 4.0, 3.0, 3.0000001, 1.0, 0.5, 0.1])
+    forced = [0, 8]
+    st = oracle.compare_index_sets([0, 1, 2, 5, 8], forced, cand, scores, 3)
+    assert st == "MISMATCH: a clearly lower candidate was kept", st
+    assert oracle.compare_index_sets([0, 1, 2, 3, 8], forced, cand, scores, 3) == "ambiguous"
+    near = scores.copy()
+    near[4] = 3.0 * (1 - 0.5e-4)          # id 5 within 1e-4 of the (k+1)-th score: still a near tie
+    assert oracle.compare_index_sets([0, 1, 2, 5, 8], forced, cand, near, 3) == "ambiguous"
+    far = scores.copy()
+    far[4] = 3.0 * (1 - 1.5e-4)           # id 5 just outside the bound
+    st = oracle.compare_index_sets([0, 1, 2, 5, 8], forced, cand, far, 3)
+    assert st == "MISMATCH: a clearly lower candidate was kept", st
+    st = oracle.compare_index_sets([0, 2, 1, 4, 8], forced, cand, scores, 3)
+    assert st == "MISMATCH: not strictly ascending", st
+    st = oracle.compare_index_sets([0, 1, 1, 4, 8], forced, cand, scores, 3)
+    assert st == "MISMATCH: not strictly ascending", st
+    st = oracle.compare_index_sets([0, 1, 2, 8, 9], forced, cand, scores, 3)
+    assert st == "MISMATCH: an id outside the candidates", st
+    # negative scores: "clearly lower" is sign-aware (-3.0 is the (k+1)-th score)
+    neg = -scores[::-1].copy()            # ids 1..7 score -0.1, -0.5, -1, -3.0000001, -3, -4, -5
+    assert oracle.compare_index_sets([0, 1, 2, 3, 5, 8], forced, cand, neg, 4) == "exact"
+    assert oracle.compare_index_sets([0, 1, 2, 3, 4, 8], forced, cand, neg, 4) == "ambiguous"
+    st = oracle.compare_index_sets([0, 1, 2, 3, 6, 8], forced, cand, neg, 4)
+    assert st == "MISMATCH: a clearly lower candidate was kept", st
+
+
 # ---------------------------------------------------------------- A-shape
 
 def test_a_shape_closed_form():

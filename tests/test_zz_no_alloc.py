@@ -22,13 +22,17 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def test_static_scratch_decode_matches_workspace_decode():
+@pytest.mark.parametrize("d,Hq,Hkv", [(128, 32, 8), (64, 16, 8), (128, 8, 1)])
+def test_static_scratch_decode_matches_workspace_decode(d, Hq, Hkv):
+    """Two calls in a row through the C ABI, each against the workspace decode
+    on the same inputs: outputs within the decode's tolerance, selections bit
+    for bit (head dims 64 and 128; GQA groups of 4, 2 and 8)."""
     assert torch.cuda.is_available()
     lib = dsa.load_library()
-    B, Hq, Hkv, S, d, keep = 4, 32, 8, 16384, 128, 64
+    B, S, keep = 4, 16384, 64
     kcap = keep + 1
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    for call, seed in enumerate((101, 202)):
+    for call, seed in enumerate((101 + d + Hq, 202 + d + Hq)):
         w = synth.make_decode("decode-b16-128k", device="cuda", B=B, S=S, Hq=Hq, Hkv=Hkv, d=d, seed=seed)
         cent = dsa.pool_keys(w.k_cache)
         ref_o, ref_si, ref_sc = dsa.sparse_decode_attn(w.q, w.k_cache, w.v_cache, cent, keep=keep, return_sel=True)
@@ -43,6 +47,20 @@ def test_static_scratch_decode_matches_workspace_decode():
         err = (o.float() - ref_o.float()).abs()
         assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3, (call, err.max().item())
         assert torch.equal(si, ref_si) and torch.equal(sc, ref_sc), call
+
+
+def test_static_scratch_decode_without_selection_outputs():
+    """The Python wrapper, with no selection outputs requested (sel_idx and
+    sel_cnt passed as NULL), twice in a row."""
+    B, Hq, Hkv, S, d, keep = 2, 32, 8, 8192, 128, 40
+    for seed in (303, 404):
+        w = synth.make_decode("decode-b16-128k", device="cuda", B=B, S=S, Hq=Hq, Hkv=Hkv, d=d, seed=seed)
+        cent = dsa.pool_keys(w.k_cache)
+        ref = dsa.sparse_decode_attn(w.q, w.k_cache, w.v_cache, cent, keep=keep)
+        got = dsa.sparse_decode_attn_static(w.q, w.k_cache, w.v_cache, cent, keep=keep)
+        torch.cuda.synchronize()
+        err = (got.float() - ref.float()).abs()
+        assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3, seed
 
 
 def test_static_scratch_rejects_oversized_problems():
