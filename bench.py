@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-decode] [--no-vs] [--no-e2e] [--no-cpu-baseline]
+                    [--no-layers] [--sustained-s S]
 
 A step is one prefill layer of the block-sparse path on the named workload
 (default: the LLaMA-3-8B-shaped layer at 128K tokens, 32 q-heads / 8 KV
@@ -11,7 +12,11 @@ index (sparse_index_estimate) followed by causal block-sparse attention
 effective TFLOP/s counting only the FLOPs of the selected blocks (diagonal
 blocks at their causal 2080 of 4096 elements); ms_per_step is ms per layer.
 The sparse decode GB/s (batch 16, 128K cache, keep 512 + the last block) is
-reported beside it under "decode".
+reported beside it under "decode", the vertical-slash layer under
+"vertical_slash", and the 32K and 1M block-sparse layers under "layers".
+"roofline" holds the attention kernel against the burst tensor peak (a few
+launches timed back to back); "roofline_sustained" the same kernel launched
+back to back for a few seconds against the sustained peak.
 
 One JSON line is printed by rank 0.  Multi-GPU (torchrun): every rank runs its
 own independent layer (weak scaling, no data-path collective); timing is the
@@ -39,13 +44,21 @@ if ROOT not in sys.path:
 
 import synth  # noqa: E402
 
-# DRAM bytes (read + write) of one bsa_fwd_kernel launch, measured with ncu
-# (dram__bytes_read.sum + dram__bytes_write.sum) on this bench's own command
-# for the workload; None for workloads without such a capture.
-BSA_TRAFFIC = {"llama3-8b-128k-bs10": 6.57e9, "llama3-8b-32k-bs10": 7.096e8}
-METRIC = "block-sparse prefill effective TFLOP/s at 128K (selected-block FLOPs)"
+# DRAM bytes (read + write) of one bsa_fwd_kernel launch, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum) of this bench's command, kept
+# with the kernel revision they were taken on (profiles/ holds the summary);
+# the line reports null for any other revision or workload.
+BSA_KERNEL_REVISION = "tile-skip-1"
+BSA_TRAFFIC = {}   # {(revision, workload): bytes}
 UNIT = "TFLOP/s"
 DIAG_ELEMS = 64 * 65 // 2
+
+
+def metric_name(workload: str) -> str:
+    """The headline metric, named for the workload's sequence length."""
+    n = synth.CONFIGS[workload]["n"]
+    label = f"{n // (1 << 20)}M" if n >= (1 << 20) else f"{n // 1024}K"
+    return f"block-sparse prefill effective TFLOP/s at {label} (selected-block FLOPs)"
 
 
 def prefill_flops(block_cnt: torch.Tensor, d: int) -> float:
@@ -268,25 +281,17 @@ def run_ours(args, rank, world, local):
     value = flops * world / (ms * 1e-3) / 1e12
     peaks, src = load_peaks()
     achieved = flops / (attn_ms * 1e-3) / 1e12
-    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    # the attention above is timed over a few back-to-back launches (well under
+    # a second): the burst peak applies.  A seconds-long run of the same kernel,
+    # held against the sustained peak, is reported beside it.
+    peak = peaks["bf16_tflops"]
+    sustained = sustained_attention(dsa, w, bi, bc, o, ws, stream, flops, peaks, seconds=args.sustained_s)
     density = float(bc.to(torch.float64).sum().item()) / (Hq * (n // 64) * (n // 64 + 1) / 2)
-    # index estimation: algorithmic bytes = Q and K read once (bf16) and the
-    # block lists written once.  The pooled scores (2*d FLOP per causal block
-    # pair, three FP16 tensor-core products of the split means, recomputed per selection pass on
-    # chip) and the per-row selection ride on that traffic; the whole call is
-    # held against the HBM copy peak.
-    nqb = n // 64
-    idx_bytes = (Hq + w.k.shape[0]) * n * d * 2 + Hq * nqb * (kcap + 1) * 4
-    idx_flops = 2.0 * d * Hq * nqb * (nqb + 1) / 2
-    idx_gbs = idx_bytes / (index_ms * 1e-3) / 1e9
-    index_roof = {"kernels": "pool_blocks (K, Q) + block_topk + block_list", "bound": "hbm",
-                  "achieved": round(idx_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                  "frac": round(idx_gbs / peaks["hbm_gbs"], 4), "bytes": idx_bytes,
-                  "score_flops": idx_flops, "score_fp16_split_products": 3}
+    index_roof = index_roofline(w, kcap, index_ms, peaks)
     res = {
-        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "metric": metric_name(args.workload), "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(args.workload, world), selected_block_density=round(density, 5)),
         "breakdown_ms": {"index": round(index_ms, 4), "attention": round(attn_ms, 4)},
         "index_roofline": index_roof,
@@ -294,14 +299,119 @@ def run_ours(args, rank, world, local):
         "effective_flops_per_step": flops,
         "roofline": {"bound": "tensor", "kernel": "bsa_fwd_kernel<128>", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": BSA_TRAFFIC.get(args.workload),
-                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch",
-                     "peak_source": f"{src} bf16_tflops_sustained"},
+                     "traffic": BSA_TRAFFIC.get((BSA_KERNEL_REVISION, args.workload)),
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch of this "
+                                       f"kernel revision ({BSA_KERNEL_REVISION})",
+                     "peak_source": f"{src} bf16_tflops (burst: {reps} launches timed back to back)",
+                     "timed_launches": reps},
+        "roofline_sustained": sustained,
         "clocks": clk.summary(),
         "gpu_launches": (launches_per_step * args.steps) if launches_per_step else None,
         "device_status": status,
     }
     return res, (w, bi, bc, kf, rho, kcap, flops, ws)
+
+
+def index_roofline(w, kcap, index_ms, peaks):
+    """The block index call held against the HBM copy peak (algorithmic bytes:
+    Q and K read once as bf16, the lists written once) and, for its scoring,
+    against the tensor peak (FP16 products issued: one per approximate pass,
+    three per exact pass, 2*d FLOP per causal (query block, key block) pair;
+    the statistics pass of long rows reads every 4th key chunk)."""
+    Hq, n, d = w.q.shape
+    nqb = n // 64
+    pairs = Hq * nqb * (nqb + 1) / 2
+    idx_bytes = (Hq + w.k.shape[0]) * n * d * 2 + Hq * nqb * (kcap + 1) * 4
+    stats_share = 1.0 if nqb <= 512 else 0.25
+    tensor_flops = 2.0 * d * pairs * (stats_share + 1 + 3)
+    gbs = idx_bytes / (index_ms * 1e-3) / 1e9
+    tfs = tensor_flops / (index_ms * 1e-3) / 1e12
+    return {"kernels": "pool_blocks (K, Q) + block_topk + block_list", "bound": "hbm", "achieved": round(gbs, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": idx_bytes,
+            "score_flops": 2.0 * d * pairs, "score_fp16_split_products": 3,
+            "tensor": {"flops_issued": tensor_flops, "achieved_tflops": round(tfs, 1), "peak": peaks["bf16_tflops"],
+                       "frac": round(tfs / peaks["bf16_tflops"], 4),
+                       "note": "FP16 kind::f16 products, same rate as bf16"}}
+
+
+def sustained_attention(dsa, w, bi, bc, o, ws, stream, flops, peaks, seconds):
+    """The attention launched back to back for about `seconds` (a long step: the
+    sustained peak applies), timed with CUDA events on its stream."""
+    if seconds <= 0:
+        return None
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    dsa.block_sparse_attn_fwd(w.q, w.k, w.v, bi, bc, out=o, ws=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = max(2, int(seconds * 1e3 / max(e0.elapsed_time(e1), 1e-3)))
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(launches):
+            dsa.block_sparse_attn_fwd(w.q, w.k, w.v, bi, bc, out=o, ws=ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / launches
+    tf = flops / (ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    return {"launches": launches, "seconds": round(ms * launches / 1e3, 2), "ms": round(ms, 4),
+            "achieved": round(tf, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(tf / peak, 4),
+            "peak_source": "bf16_tflops_sustained", "clocks": clk.summary()}
+
+
+def run_layers(args, local, names):
+    """The other block-sparse prefill layers (index + attention each), for the
+    workloads' own sizes: ms per layer, effective TFLOP/s of the attention
+    against the tensor peak, and the index against HBM (and, for its scoring,
+    the tensor peak)."""
+    import dynamic_sparse_attention_03_b200 as dsa
+
+    dev = torch.device("cuda", local)
+    peaks, src = load_peaks()
+    out = {}
+    for name in names:
+        p = synth.CONFIGS[name]
+        w = synth.make_prefill(name, device=dev)
+        Hq, n, d = w.q.shape
+        kf, rho = p.get("k_fixed", 0), p.get("keep_ratio", 0.0)
+        kcap = dsa.block_index_capacity(n, kf, rho)
+        bi = torch.empty((Hq, n // 64, kcap), dtype=torch.int32, device=dev)
+        bc = torch.empty((Hq, n // 64), dtype=torch.int32, device=dev)
+        o = torch.empty_like(w.q)
+        ws = dsa.Workspace(dev)
+        stream = torch.cuda.current_stream(dev)
+        reps = 2 if n > 200000 else 5
+        for _ in range(2):
+            dsa.sparse_index_estimate(w.q, w.k, k_fixed=kf, keep_ratio=rho, kcap=kcap, block_idx=bi, block_cnt=bc,
+                                      ws=ws)
+            dsa.block_sparse_attn_fwd(w.q, w.k, w.v, bi, bc, out=o, ws=ws)
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        for _ in range(reps):
+            dsa.sparse_index_estimate(w.q, w.k, k_fixed=kf, keep_ratio=rho, kcap=kcap, block_idx=bi, block_cnt=bc,
+                                      ws=ws)
+        ev[1].record(stream)
+        for _ in range(reps):
+            dsa.block_sparse_attn_fwd(w.q, w.k, w.v, bi, bc, out=o, ws=ws)
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        index_ms = ev[0].elapsed_time(ev[1]) / reps
+        attn_ms = ev[1].elapsed_time(ev[2]) / reps
+        flops = prefill_flops(bc, d)
+        tf = flops / (attn_ms * 1e-3) / 1e12
+        density = float(bc.to(torch.float64).sum().item()) / (Hq * (n // 64) * (n // 64 + 1) / 2)
+        out[name] = {"index_ms": round(index_ms, 4), "attention_ms": round(attn_ms, 4),
+                     "ms_per_layer": round(index_ms + attn_ms, 4), "effective_flops": flops,
+                     "effective_tflops_attention": round(tf, 1),
+                     "frac_attention": round(tf / peaks["bf16_tflops"], 4),
+                     "peak_attention": peaks["bf16_tflops"], "peak_source": f"{src} bf16_tflops (burst)",
+                     "selected_block_density": round(density, 5), "index_roofline": index_roofline(w, kcap, index_ms,
+                                                                                                    peaks),
+                     "timed_launches": reps, "status": dsa.get_status(ws)}
+        del w, bi, bc, o, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_dense(args, ctx, local, attn_flops_ms):
@@ -497,11 +607,25 @@ def run_vs(args, local):
     flops = prefill_flops(res["block_cnt"], d) + float(res["col_cnt"].to(torch.float64).sum().item()) * 4 * d * 64
     nqb = n // 64
     density = float(res["block_cnt"].to(torch.float64).sum().item()) / (Hq * nqb * (nqb + 1) / 2)
-    peaks, _ = load_peaks()
+    peaks, src = load_peaks()
     tf = flops / (att_ms * 1e-3) / 1e12
+    # the index: K read once (bf16) and the last 64 query rows, the kept sets
+    # and the plan's lists written once; 2 x 2*64*n*d FLOP of logits per q-head
+    # (the scores' pass and the sums' pass) on the tensor pipe
+    Hkv = w.k.shape[0]
+    kcap, ccap = res["block_idx"].shape[-1], res["col_idx"].shape[-1]
+    idx_bytes = (Hkv * n * d + Hq * 64 * d) * 2 + Hq * (p["n_vert"] + p["n_slash"]) * 4 + \
+        Hq * nqb * (kcap + ccap + 2) * 4
+    idx_flops = 2 * 2.0 * 64 * n * d * Hq
+    gbs = idx_bytes / (idx_ms * 1e-3) / 1e9
+    tfs = idx_flops / (idx_ms * 1e-3) / 1e12
     out = {"workload": name, "index_ms": round(idx_ms, 3), "attention_ms": round(att_ms, 3),
            "ms_per_layer": round(idx_ms + att_ms, 3), "effective_tflops_attention": round(tf, 1),
-           "frac_attention": round(tf / peaks.get("bf16_tflops_sustained", 1362.1), 4),
+           "frac_attention": round(tf / peaks["bf16_tflops"], 4), "peak_source": f"{src} bf16_tflops (burst)",
+           "index_roofline": {"bound": "hbm", "bytes": idx_bytes, "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                              "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                              "tensor_flops": idx_flops, "achieved_tflops": round(tfs, 1),
+                              "tensor_frac": round(tfs / peaks["bf16_tflops"], 4)},
            "selected_block_density": round(density, 4), "status": dsa.get_status(ws)}
     del w, res, o
     torch.cuda.empty_cache()
@@ -617,6 +741,17 @@ def oracle_sample(workload: str, budget_s: float, w=None, seed_rank: int = 0):
     return flops / t_total / 1e12, desc, t_total, cores
 
 
+def blas_threads():
+    """Threads of the BLAS library NumPy's matrix products use (None if unknown)."""
+    try:
+        import threadpoolctl
+
+        info = [x for x in threadpoolctl.threadpool_info() if x.get("user_api") == "blas"]
+        return info[0]["num_threads"] if info else None
+    except Exception:
+        return None
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -632,11 +767,12 @@ def run_reference(args, rank, world):
         if i >= args.warmup:
             vals.append(v)
     value = statistics.mean(vals)
-    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+    return {"metric": metric_name(args.workload), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": workload_config(args.workload, world),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "blas_threads": blas_threads(),
+                             "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -653,6 +789,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-layers", action="store_true", help="skip the 32K and 1M layers")
+    ap.add_argument("--sustained-s", type=float, default=3.0,
+                    help="seconds of back-to-back attention launches for the sustained-peak line (0: skip)")
     ap.add_argument("--decode-batch", type=int, default=16,
                     help="batch of the decode workloads (16 is the reported configuration; smaller for profiling)")
     args = ap.parse_args()
@@ -671,6 +810,9 @@ def main():
         res["e2e"] = run_e2e(args, ctx, local)
     if not args.no_dense:
         res["dense_comparator"] = run_dense(args, ctx, local, res["breakdown_ms"]["attention"])
+    if not args.no_layers:
+        others = [x for x in ("llama3-8b-32k-bs10", "llama3-8b-1m-bs2") if x != args.workload]
+        res["layers"] = run_layers(args, local, others)
     if not args.no_decode:
         res["decode"] = run_decode(args, local)
     if not args.no_clusters:
@@ -679,8 +821,8 @@ def main():
         res["vertical_slash"] = run_vs(args, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, secs, cores = oracle_sample(args.workload, 15.0, w=ctx[0])
-        res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
-                               "seconds": round(secs, 2)}
+        res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "blas_threads": blas_threads(),
+                               "kind": "oracle", "sample": desc, "seconds": round(secs, 2)}
     if world > 1:
         import torch.distributed as dist
 

@@ -101,6 +101,15 @@ bool validate_env() {
   return v && v[0] == '1';
 }
 
+// Fault injection for the tests of the bounded waits: with
+// DSA_FAULT_INJECT=attn_stall, block_sparse_attn_fwd's first work item issues
+// no load for its first K tile and the waits give up after 1 ms, so the call
+// ends with DSA_ERR_TIMEOUT in the status word and nothing in flight.
+bool stall_injection() {
+  const char* v = std::getenv("DSA_FAULT_INJECT");
+  return v && std::strcmp(v, "attn_stall") == 0;
+}
+
 int max_count(int nQB, int k_fixed, int64_t ppm) {
   int best = 0;
   for (int i = 0; i < nQB; ++i) {
@@ -166,6 +175,12 @@ int launch_attn(const void* q, const void* k, const void* v, void* o, int Hq, in
   p.grp = Hq / Hkv;
   p.nquads = (p.grp + 3) / 4;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_ns = kWaitLimitNs;
+  p.stall_item = -1;
+  if (stall_injection()) {   // test hook: one K load is skipped, its wait runs out after 1 ms
+    p.wait_ns = 1000000ull;
+    p.stall_item = 0;
+  }
   const size_t smem = AttnLayout<D>::kSmemAlloc;
   int rc = set_smem(bsa_fwd_kernel<D>, smem);
   if (rc) return rc;

@@ -20,21 +20,27 @@
 //    products have.
 //  * Warp 1 walks the MMA schedule warp-uniformly (one elected lane issues),
 //    in the order QK_A(t+1), PV_B(t), QK_B(t+1), PV_A(t+1), ...:
-//    S = Q K^T (M=128, N=128, K=d, shared-memory
-//    operands) into TMEM S_A / S_B, and O += P V (M=128, N=d, K=128) with P
-//    read from TMEM (aliased onto the first 64 columns of S) and V from shared
-//    memory.  tcgen05.mma operations of a CTA run in issue order, so the PV
-//    that reads P(t) finishes before the next QK^T overwrites S.  While one
-//    softmax warpgroup works on its tile, the tensor pipe runs the other
-//    tile's products.
+//    S = Q K^T (M=128, shared-memory operands) into TMEM S_A / S_B, and
+//    O += P V (M=128, N=d) with P read from TMEM (aliased onto the first 64
+//    columns of S) and V from shared memory.  A query tile's products cover
+//    only the slots one of its two heads chose: both slots (N=128), one slot
+//    (N=64 QK^T, K=64 PV), or none (the tile skips that step; its barriers
+//    count processed steps, so the issuer and the softmax warps, which both
+//    decide from the step's metadata, stay in phase).  tcgen05.mma operations
+//    of a CTA run in issue order, so the PV that reads P(t) finishes before
+//    the next QK^T overwrites S.  While one softmax warpgroup works on its
+//    tile, the tensor pipe runs the other tile's products.
 //  * Warps 4-7 (tile A) and 8-11 (tile B) run the online softmax, one row per
-//    thread (= TMEM lane): a first pass over the S row for the max, a second
-//    for exp2(s*scale*log2e - max) with packed f32x2 FMAs, P (bf16) written
-//    back into TMEM with tcgen05.st, a lazy rescale of O in TMEM only when the
-//    running max grows by more than 2^8, and the epilogue O / l -> bf16.
+//    thread (= TMEM lane): the row max over the visible keys, then
+//    exp2(s*scale*log2e - max) with packed f32x2 FMAs, P (bf16) written back
+//    into TMEM with tcgen05.st, a lazy rescale of O in TMEM only when the
+//    running max grows by more than 2^8, and the epilogue O / l -> bf16.  A
+//    slot that the row's head did not choose costs no exponentials (its P is
+//    zero, written only if the other head of the tile chose it).
 //  * TMEM columns: S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512).
-//  * Every wait is bounded (1 s); on expiry the CTA records a timeout in the
-//    status word, all roles leave their loops, TMEM is freed, the CTA returns.
+//  * Every wait is bounded (1 s, or the caller's limit); on expiry the CTA
+//    records a timeout in the status word, all roles leave their loops, TMEM is
+//    freed, the CTA returns.
 #pragma once
 
 #include <cuda.h>
@@ -58,6 +64,8 @@ struct AttnParams {
   int kcap, ccap;
   int Hq, Hkv, n, nQB, grp, nquads;
   float scale_log2;
+  uint64_t wait_ns;   // bounded-wait limit
+  int stall_item;     // test hook: this work item skips its first K load (-1: none)
 };
 
 // Per-tile metadata for the MMA issuer and the softmax warpgroups.
@@ -117,6 +125,16 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, u
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
       "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Writes 32 columns of zeros (32 lanes x 32 columns) at taddr.
+__device__ __forceinline__ void tmem_st32_zero(uint32_t taddr) {
+  const uint32_t z = 0u;
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr), "r"(z)
       : "memory");
 }
 
@@ -269,11 +287,14 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const AbortState ab{abort_flag, p.status};
+  const AbortState ab{abort_flag, p.status, p.wait_ns};
 
   auto sQ = [&](int tile) { return sb + (tile ? Lay::kQB : Lay::kQA); };
   auto sK = [&](int s) { return sb + Lay::kK0 + (uint32_t)s * Lay::kTile; };
   auto sV = [&](int s) { return sb + Lay::kV0 + (uint32_t)s * Lay::kTile; };
+  // slot s of a step is computed for query tile X (heads 2X, 2X+1 of the item)
+  // when one of those heads chose it
+  auto vis = [](const AttnMeta& M, int X, int s) { return (M.m[s][2 * X] | M.m[s][2 * X + 1]) != 0ull; };
 
   if (warp == 0 || warp == 2) {
     // ------------------------------------------------------------ producers
@@ -308,6 +329,9 @@ __global__ void __launch_bounds__(384, 1)
     const __nv_bfloat16* base = (isK ? p.k : p.v) + (size_t)g * p.n * D;
     int(*cols)[64] = isK ? colsK : colsV;
     const int full0 = isK ? AB_KFULL : AB_VFULL, empty0 = isK ? AB_KEMPTY : AB_VEMPTY;
+    // test hook: the K producer of work item stall_item issues nothing for its
+    // first tile, so the MMA warp's wait for it runs out (nothing is in flight)
+    const int skipped = (isK && p.stall_item == (int)blockIdx.x) ? 0 : -1;
     int t = 0, issued = 0;
     while (true) {
       const int s = t % NS;
@@ -326,25 +350,28 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) {
         if (isK) mbar_arrive(bar(AB_META + (t % kAttnMR)));
-        const uint32_t tx = (uint32_t)((k0 == 1) + (k1 == 1)) * 64u * D * 2u;
-        mbar_arrive_expect_tx(bar(full0 + s), tx);
-        if (k0 == 1)
+        if (t != skipped) {
+          const uint32_t tx = (uint32_t)((k0 == 1) + (k1 == 1)) * 64u * D * 2u;
+          mbar_arrive_expect_tx(bar(full0 + s), tx);
+          if (k0 == 1)
 #pragma unroll
-          for (int dh = 0; dh < Lay::NDH; ++dh)
-            tma_load_2d(stg + dh * Lay::kHalf, tm, dh * 64, g * p.n + b0 * 64, bar(full0 + s));
-        if (k1 == 1)
+            for (int dh = 0; dh < Lay::NDH; ++dh)
+              tma_load_2d(stg + dh * Lay::kHalf, tm, dh * 64, g * p.n + b0 * 64, bar(full0 + s));
+          if (k1 == 1)
 #pragma unroll
-          for (int dh = 0; dh < Lay::NDH; ++dh)
-            tma_load_2d(stg + dh * Lay::kHalf + 8192, tm, dh * 64, g * p.n + b1 * 64, bar(full0 + s));
+            for (int dh = 0; dh < Lay::NDH; ++dh)
+              tma_load_2d(stg + dh * Lay::kHalf + 8192, tm, dh * 64, g * p.n + b1 * 64, bar(full0 + s));
+        }
       }
       __syncwarp();
       ++issued;
       if (nsl == 0 || last) break;
       ++t;
     }
+    // wait for this producer's own copies still in flight (none for a skipped tile)
     if (lane == 0) {
       for (int u = max(0, issued - NS); u < issued; ++u)
-        mbar_wait_cleanup(bar(full0 + (u % NS)), (u / NS) & 1, 200000000ull);
+        if (u != skipped) mbar_wait_cleanup(bar(full0 + (u % NS)), (u / NS) & 1, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -360,77 +387,112 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t dQ0 = umma_desc_sw128(sQ(0), 16, 1024), dQ1 = umma_desc_sw128(sQ(1), 16, 1024);
     const uint64_t dK0 = umma_desc_sw128(sK(0), 16, 1024);
     const uint64_t dV0 = umma_desc_sw128(sV(0), Lay::kHalf, 1024);
-    auto qk = [&](int tile, int ks, int nsl) {
-      const uint32_t idesc = nsl > 1 ? idesc_qk2 : idesc_qk1;
-      const uint32_t dS = tmem + kTmemS + 128u * (uint32_t)tile;
-      const uint64_t a0 = tile ? dQ1 : dQ0;
-      const uint64_t b0 = dK0 + (uint64_t)(((uint32_t)ks * (uint32_t)Lay::kTile) >> 4);
+    // S_X = Q_X K^T over the chosen slots v0 / v1 of K stage ks (key rows
+    // 64..127 of a stage start 8192 bytes into each d-half)
+    auto qk = [&](int X, int ks, bool v0, bool v1) {
+      const uint32_t idesc = (v0 && v1) ? idesc_qk2 : idesc_qk1;
+      const uint32_t first = v0 ? 0u : 1u;
+      const uint32_t dS = tmem + kTmemS + 128u * (uint32_t)X + 64u * first;
+      const uint64_t a0 = X ? dQ1 : dQ0;
+      const uint64_t b0 = dK0 + (uint64_t)(((uint32_t)ks * (uint32_t)Lay::kTile + 8192u * first) >> 4);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = (uint64_t)(((kk >> 2) * Lay::kHalf + (kk & 3) * 32) >> 4);
         if (issuer) umma_bf16_ss(dS, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
       }
-      if (issuer) umma_commit(bar(AB_SFULL + tile));
+      if (issuer) umma_commit(bar(AB_SFULL + X));
     };
-    auto pv = [&](int tile, int u, int nsl) {
+    // O_X += P_X V over the chosen slots of V stage u; the first product of the
+    // item into O_X starts the accumulator
+    bool acc[2] = {false, false};
+    auto pv = [&](int X, int u, bool v0, bool v1) {
       const uint64_t b0 = dV0 + (uint64_t)(((uint32_t)(u % kAttnVS) * (uint32_t)Lay::kTile) >> 4);
-      const uint32_t pa = tmem + kTmemS + 128u * (uint32_t)tile;   // P aliases the first 64 columns of S
-      const uint32_t dO = tmem + kTmemO + 128u * (uint32_t)tile;
+      const uint32_t pa = tmem + kTmemS + 128u * (uint32_t)X;   // P aliases the first 64 columns of S
+      const uint32_t dO = tmem + kTmemO + 128u * (uint32_t)X;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        if (kk < nsl * 4 && issuer)
-          umma_bf16_ts(dO, pa + 8u * (uint32_t)kk, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv,
-                       (u > 0 || kk > 0) ? 1u : 0u);
+        if (kk < 4 ? v0 : v1) {
+          if (issuer) umma_bf16_ts(dO, pa + 8u * (uint32_t)kk, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                                   acc[X] ? 1u : 0u);
+          acc[X] = true;
+        }
       }
-      if (issuer) umma_commit(bar(AB_PVDONE + tile));
     };
     bool ok = mbar_wait_warp(bar(AB_Q), 0, ab);
-    int t = 0;
-    int nsl = 0, last = 1;
+    int t = 0, last = 1;
+    bool done[2] = {false, false};   // the epilogue's arrival on PVDONE_X was committed
+    int nP[2] = {0, 0};   // P phases consumed per query tile
+    bool cv[2][2] = {{false, false}, {false, false}};   // chosen slots of step t per tile
     if (ok) ok = mbar_wait_warp(bar(AB_KFULL), 0, ab);
     if (ok) {
-      nsl = meta[0].nslots;
-      last = meta[0].last;
-      if (nsl > 0) {
+      const AttnMeta& M = meta[0];
+      last = M.last;
+      if (M.nslots > 0) {
         tc_fence_after();
-        qk(0, 0, nsl);
-        if (hasB) qk(1, 0, nsl);
+#pragma unroll
+        for (int X = 0; X < 2; ++X) {
+          cv[X][0] = (X == 0 || hasB) && vis(M, X, 0);
+          cv[X][1] = (X == 0 || hasB) && vis(M, X, 1);
+          if (cv[X][0] || cv[X][1]) qk(X, 0, cv[X][0], cv[X][1]);
+        }
         if (issuer) umma_commit(bar(AB_KEMPTY));
+      } else {
+        ok = false;
       }
     }
-    while (ok && nsl > 0) {
-      int nsl_next = 0, last_next = 1;
-      // PV_A(t) ; QK_A(t+1).  The operand tiles usually land before P does,
-      // so their waits come first and P_A(t) is consumed as soon as it is ready.
+    while (ok) {
+      // PV_X(t) ; QK_X(t+1) for X = A, B.  The operand tiles usually land
+      // before P does, so their waits come first.
+      bool nv[2][2] = {{false, false}, {false, false}};
+      int last_next = 1;
       const int ks = (t + 1) % kAttnKS;
-      if (!mbar_wait_warp(bar(AB_VFULL + (t % kAttnVS)), (t / kAttnVS) & 1, ab)) { ok = false; break; }
+      if (!mbar_wait_warp(bar(AB_VFULL + (t % kAttnVS)), (t / kAttnVS) & 1, ab)) break;
       if (!last) {
-        if (!mbar_wait_warp(bar(AB_KFULL + ks), ((t + 1) / kAttnKS) & 1, ab)) { ok = false; break; }
-        nsl_next = meta[(t + 1) % kAttnMR].nslots;
-        last_next = meta[(t + 1) % kAttnMR].last;
+        if (!mbar_wait_warp(bar(AB_KFULL + ks), ((t + 1) / kAttnKS) & 1, ab)) break;
+        const AttnMeta& M = meta[(t + 1) % kAttnMR];
+        last_next = M.last;
+#pragma unroll
+        for (int X = 0; X < 2; ++X) {
+          nv[X][0] = (X == 0 || hasB) && vis(M, X, 0);
+          nv[X][1] = (X == 0 || hasB) && vis(M, X, 1);
+        }
       }
-      if (!mbar_wait_warp(bar(AB_PFULL + 0), t & 1, ab)) { ok = false; break; }
-      tc_fence_after();
-      pv(0, t, nsl);
-      if (!last) qk(0, ks, nsl_next);
-      // PV_B(t) ; QK_B(t+1)
-      if (hasB) {
-        if (!mbar_wait_warp(bar(AB_PFULL + 1), t & 1, ab)) { ok = false; break; }
-        tc_fence_after();
-        pv(1, t, nsl);
-        if (!last) qk(1, (t + 1) % kAttnKS, nsl_next);
+      bool stop = false;
+#pragma unroll
+      for (int X = 0; X < 2; ++X) {   // unrolled: X is a constant, the per-tile flags stay in registers
+        if (!stop && (cv[X][0] || cv[X][1])) {
+          if (!mbar_wait_warp(bar(AB_PFULL + X), nP[X] & 1, ab)) {
+            stop = true;
+          } else {
+            ++nP[X];
+            tc_fence_after();
+            pv(X, t, cv[X][0], cv[X][1]);
+            if (last && issuer) umma_commit(bar(AB_PVDONE + X));   // O_X is final once this completes
+            done[X] = done[X] || last;
+          }
+        }
+        if (!stop && !last && (nv[X][0] || nv[X][1])) qk(X, ks, nv[X][0], nv[X][1]);
       }
+      if (stop) break;
       if (issuer) {
         umma_commit(bar(AB_VEMPTY + (t % kAttnVS)));
-        if (!last) umma_commit(bar(AB_KEMPTY + ((t + 1) % kAttnKS)));
+        if (!last) umma_commit(bar(AB_KEMPTY + ks));
       }
       if (last) break;
-      nsl = nsl_next;
+#pragma unroll
+      for (int X = 0; X < 2; ++X) {
+        cv[X][0] = nv[X][0];
+        cv[X][1] = nv[X][1];
+      }
       last = last_next;
       ++t;
     }
-    // Drain: every MMA of this CTA has completed before TMEM is freed.
+    // One arrival per query tile on PVDONE (a tile that did not compute the
+    // last step, or an aborted run, gets it here), and every MMA of this CTA
+    // has completed before TMEM is freed.
     if (issuer) {
+      if (!done[0]) umma_commit(bar(AB_PVDONE + 0));
+      if (!done[1]) umma_commit(bar(AB_PVDONE + 1));
       umma_commit(bar(AB_DRAIN));
       mbar_wait_cleanup(bar(AB_DRAIN), 0, 200000000ull);
     }
@@ -440,7 +502,7 @@ __global__ void __launch_bounds__(384, 1)
     const int tile = (warp - 4) >> 2;     // 0: warps 4-7, 1: warps 8-11
     const int q4 = warp & 3;              // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;
-    const int hh = 2 * tile + (row >> 6);  // head of the item for this row
+    const int hh = 2 * tile + (row >> 6);  // head of the item for this row (warp-uniform)
     const int r = row & 63;
     const bool active = (tile == 0) || hasB;
     const uint32_t laddr = tmem + ((uint32_t)(q4 * 32) << 16);
@@ -449,32 +511,35 @@ __global__ void __launch_bounds__(384, 1)
     const unsigned long long causal = (r == 63) ? ~0ull : ((1ull << (r + 1)) - 1ull);
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
-    int t = 0;
-    bool ok = true, any = false;
+    int t = 0, nS = 0;   // steps seen; S phases consumed (steps this tile computed)
+    bool ok = true;
     while (active) {
       if (!mbar_wait_warp(bar(AB_META + (t % kAttnMR)), (t / kAttnMR) & 1, ab)) { ok = false; break; }
       const AttnMeta& M = meta[t % kAttnMR];
       const int nsl = M.nslots;
       if (nsl == 0) break;
       const int last = M.last;
-      unsigned long long vm0 = M.m[0][hh];
-      if (M.kind[0] == 1 && M.blk[0] == qb) vm0 &= causal;
-      unsigned long long vm1 = 0ull;
-      if (nsl > 1) {
-        vm1 = M.m[1][hh];
-        if (M.kind[1] == 1 && M.blk[1] == qb) vm1 &= causal;
+      const bool c0 = vis(M, tile, 0), c1 = nsl > 1 && vis(M, tile, 1);   // slots the tile computed
+      if (!c0 && !c1) {   // neither head of this tile chose this step
+        if (last) break;
+        ++t;
+        continue;
       }
-      // Per slot and row: every key visible, none visible, or a partial mask
-      // (the diagonal block, column slots).  Warps whose rows are all "every" or
-      // "none" take the fast path: a hidden slot gets FMA scale 0 and bias
-      // -inf, so its exp2 is 0 without any per-key work.
-      const bool none0 = vm0 == 0ull, none1 = vm1 == 0ull;
-      const bool fast0 = __all_sync(0xFFFFFFFFu, none0 || vm0 == ~0ull);
-      const bool fast1 = __all_sync(0xFFFFFFFFu, none1 || vm1 == ~0ull);
-      if (!mbar_wait_warp(bar(AB_SFULL + tile), t & 1, ab)) { ok = false; break; }
+      // this row's keys per slot (warp-uniform: a warp's rows share one head)
+      unsigned long long vm0 = c0 ? M.m[0][hh] : 0ull;
+      if (M.kind[0] == 1 && M.blk[0] == qb) vm0 &= causal;
+      unsigned long long vm1 = c1 ? M.m[1][hh] : 0ull;
+      if (nsl > 1 && M.kind[1] == 1 && M.blk[1] == qb) vm1 &= causal;
+      // a slot is visible, hidden (no exponentials), or partial (the diagonal
+      // block, column slots: per-key masks)
+      const bool none0 = __all_sync(0xFFFFFFFFu, vm0 == 0ull), none1 = __all_sync(0xFFFFFFFFu, vm1 == 0ull);
+      const bool full0 = __all_sync(0xFFFFFFFFu, vm0 == ~0ull), full1 = __all_sync(0xFFFFFFFFu, vm1 == ~0ull);
+      if (!mbar_wait_warp(bar(AB_SFULL + tile), nS & 1, ab)) { ok = false; break; }
+      ++nS;
       tc_fence_after();
-      // The S row of both slots (128 keys) in registers with one TMEM round
-      // trip; hidden keys of partially visible slots are set to -inf first.
+      // the S row of both slots in registers with one TMEM round trip (a slot
+      // the tile did not compute, or that this row's head hid, is never read
+      // from these registers); hidden keys of partial slots are set to -inf
       uint32_t sv[4][32];
       tmem_ld32(sS, sv[0]);
       tmem_ld32(sS + 32, sv[1]);
@@ -487,7 +552,7 @@ __global__ void __launch_bounds__(384, 1)
       reg_fence(sv[1]);
       reg_fence(sv[2]);
       reg_fence(sv[3]);
-      if (!fast0) {
+      if (!none0 && !full0) {
         const uint32_t lo = (uint32_t)vm0, hi = (uint32_t)(vm0 >> 32);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -495,7 +560,7 @@ __global__ void __launch_bounds__(384, 1)
           sv[1][c] = ((hi >> c) & 1u) ? sv[1][c] : 0xFF800000u;
         }
       }
-      if (nsl > 1 && !fast1) {
+      if (!none1 && !full1) {
         const uint32_t lo = (uint32_t)vm1, hi = (uint32_t)(vm1 >> 32);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -504,26 +569,26 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       // row max of the raw scores over the visible keys (the scale is positive)
-      float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
+      float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
       if (!none0) {
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
-          c0 = fmax3(c0, __uint_as_float(sv[0][c]), __uint_as_float(sv[0][c + 1]));
-          c1 = fmax3(c1, __uint_as_float(sv[0][c + 2]), __uint_as_float(sv[0][c + 3]));
-          c2 = fmax3(c2, __uint_as_float(sv[1][c]), __uint_as_float(sv[1][c + 1]));
-          c3 = fmax3(c3, __uint_as_float(sv[1][c + 2]), __uint_as_float(sv[1][c + 3]));
+          x0 = fmax3(x0, __uint_as_float(sv[0][c]), __uint_as_float(sv[0][c + 1]));
+          x1 = fmax3(x1, __uint_as_float(sv[0][c + 2]), __uint_as_float(sv[0][c + 3]));
+          x2 = fmax3(x2, __uint_as_float(sv[1][c]), __uint_as_float(sv[1][c + 1]));
+          x3 = fmax3(x3, __uint_as_float(sv[1][c + 2]), __uint_as_float(sv[1][c + 3]));
         }
       }
-      if (nsl > 1 && !none1) {
+      if (!none1) {
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
-          c0 = fmax3(c0, __uint_as_float(sv[2][c]), __uint_as_float(sv[2][c + 1]));
-          c1 = fmax3(c1, __uint_as_float(sv[2][c + 2]), __uint_as_float(sv[2][c + 3]));
-          c2 = fmax3(c2, __uint_as_float(sv[3][c]), __uint_as_float(sv[3][c + 1]));
-          c3 = fmax3(c3, __uint_as_float(sv[3][c + 2]), __uint_as_float(sv[3][c + 3]));
+          x0 = fmax3(x0, __uint_as_float(sv[2][c]), __uint_as_float(sv[2][c + 1]));
+          x1 = fmax3(x1, __uint_as_float(sv[2][c + 2]), __uint_as_float(sv[2][c + 3]));
+          x2 = fmax3(x2, __uint_as_float(sv[3][c]), __uint_as_float(sv[3][c + 1]));
+          x3 = fmax3(x3, __uint_as_float(sv[3][c + 2]), __uint_as_float(sv[3][c + 3]));
         }
       }
-      const float mt = fmaxf(fmaxf(c0, c1), fmaxf(c2, c3)) * sl2;
+      const float mt = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)) * sl2;
       float m_new = m_run;
       bool rescale = false;
       if (m_run == -INFINITY) {
@@ -534,37 +599,39 @@ __global__ void __launch_bounds__(384, 1)
       }
       const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
       const float nmu = (m_new == -INFINITY) ? 0.f : -m_new;
-      // p = 2^(s*scale*log2e - m); P (bf16, two keys per 32-bit column) over the
-      // first 64 columns of S, which have all been read above.
+      // p = 2^(s*scale*log2e - m); P (bf16, two keys per 32-bit column) over
+      // the first 64 columns of S, which have all been read above.  A slot
+      // the tile computed but this row's head did not choose gets P = 0.
       float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int sl = 0; sl < 2; ++sl) {
-        if (sl >= nsl) break;
-        const bool none = sl ? none1 : none0;
-        // hidden slot: 2^(0*s - inf) = 0 on the fast path; masked keys are
-        // already -inf (and must not be multiplied by 0)
-        const float k2 = (none && (sl ? fast1 : fast0)) ? 0.f : sl2;
-        const float b2 = none ? -INFINITY : nmu;
-        uint32_t pk[32];
+        if (!(sl ? c1 : c0)) continue;
+        if (sl ? none1 : none0) {
+          tmem_st32_zero(sS + 32 * sl);
+        } else {
+          uint32_t pk[32];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float2 ea = ffma2(make_float2(__uint_as_float(sv[2 * sl][2 * j]), __uint_as_float(sv[2 * sl][2 * j + 1])),
-                                  make_float2(k2, k2), make_float2(b2, b2));
-          const float2 eb =
-              ffma2(make_float2(__uint_as_float(sv[2 * sl + 1][2 * j]), __uint_as_float(sv[2 * sl + 1][2 * j + 1])),
-                    make_float2(k2, k2), make_float2(b2, b2));
-          const float2 pa = make_float2(ex2_approx(ea.x), ex2_approx(ea.y));
-          const float2 pb = make_float2(ex2_approx(eb.x), ex2_approx(eb.y));
-          sum2 = fadd2(sum2, fadd2(pa, pb));
-          pk[j] = pack_bf16x2(pa.x, pa.y);
-          pk[16 + j] = pack_bf16x2(pb.x, pb.y);
+          for (int j = 0; j < 16; ++j) {
+            const float2 ea =
+                ffma2(make_float2(__uint_as_float(sv[2 * sl][2 * j]), __uint_as_float(sv[2 * sl][2 * j + 1])),
+                      make_float2(sl2, sl2), make_float2(nmu, nmu));
+            const float2 eb =
+                ffma2(make_float2(__uint_as_float(sv[2 * sl + 1][2 * j]), __uint_as_float(sv[2 * sl + 1][2 * j + 1])),
+                      make_float2(sl2, sl2), make_float2(nmu, nmu));
+            const float2 pa = make_float2(ex2_approx(ea.x), ex2_approx(ea.y));
+            const float2 pb = make_float2(ex2_approx(eb.x), ex2_approx(eb.y));
+            sum2 = fadd2(sum2, fadd2(pa, pb));
+            pk[j] = pack_bf16x2(pa.x, pa.y);
+            pk[16 + j] = pack_bf16x2(pb.x, pb.y);
+          }
+          tmem_st32(sS + 32 * sl, pk);
         }
-        tmem_st32(sS + 32 * sl, pk);
       }
       l_run = l_run * alpha + (sum2.x + sum2.y);
       m_run = m_new;
-      // O rescale: the PV of the previous tile has completed (it was issued
-      // before this tile's QK^T, and the tensor pipe runs in order).
+      // O rescale: the PV of the previous step has completed (it was issued
+      // before this step's QK^T, and the commit of S waits for every earlier
+      // product of the CTA).
       if (__any_sync(0xFFFFFFFFu, rescale)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -581,11 +648,11 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(AB_PFULL + tile));
-      any = true;
       if (last) break;
       ++t;
     }
-    if (active && ok && any) ok = mbar_wait_warp(bar(AB_PVDONE + tile), t & 1, ab);
+    const bool any = nS > 0;
+    if (active && ok) ok = mbar_wait_warp(bar(AB_PVDONE + tile), 0, ab);
     if (active && ok && hh < nh) {
       tc_fence_after();
       const int h = h0 + hh;

@@ -66,13 +66,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Shared abort state of one CTA: once any wait in the CTA gives up, every
 // later wait returns false at once so all roles leave their loops.
 struct AbortState {
-  volatile int* flag;   // shared memory
-  uint32_t* status;     // global status word
+  volatile int* flag;                  // shared memory
+  uint32_t* status;                    // global status word
+  uint64_t limit_ns = kWaitLimitNs;    // a wait gives up after this long
 };
 
 // Wait for the phase with the given parity to complete.  Returns false if the
-// wait gave up (time limit or the CTA is aborting); the caller must then leave
-// its loop.  The limit is checked on the global timer every 256 polls.
+// wait gave up (the time limit ab.limit_ns, or the CTA is aborting); the caller
+// must then leave its loop.  The limit is checked on the global timer every
+// 256 polls.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const AbortState& ab) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = global_timer_ns();
@@ -84,7 +86,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const A
         *ab.flag = 1;
         return false;
       }
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > ab.limit_ns) {
         *ab.flag = 1;
         atomicOr(ab.status, kStatusTimeout);
         return false;
