@@ -375,15 +375,14 @@ int vertical_slash_index(const void* q, const void* k, int Hq, int Hkv, int n, i
   if (!(scale > 0.f) || !aligned16(q) || !aligned16(k)) return DSA_ERR_INVALID_ARG;
   const int nQB = n / 64;
   if (kcap < std::min(nQB, 2 * n_slash) || ccap < n_vert) return DSA_ERR_CAPACITY;
-  const int ntiles = nQB;
+  const int ntiles = (n + kVSTile - 1) / kVSTile;
   WsCarve c(ws);
   VSParams p{};
   p.status = static_cast<uint32_t*>(c.take(kStatusBytes));
-  p.zlog = static_cast<float*>(c.take((size_t)Hq * 64 * n * 4));
   p.part = static_cast<float*>(c.take((size_t)Hq * ntiles * 64 * 2 * 4));
   p.lse2 = static_cast<float*>(c.take((size_t)Hq * 64 * 4));
   p.vert = static_cast<float*>(c.take((size_t)Hq * n * 4));
-  p.slash_part = static_cast<float*>(c.take((size_t)Hq * ntiles * 127 * 4));
+  p.slash_part = static_cast<float*>(c.take((size_t)Hq * ntiles * kVSDiag * 4));
   p.slash = static_cast<float*>(c.take((size_t)Hq * n * 4));
   p.vsel = vert_idx ? vert_idx : static_cast<int32_t*>(c.take((size_t)Hq * n_vert * 4));
   p.ssel = slash_off ? slash_off : static_cast<int32_t*>(c.take((size_t)Hq * n_slash * 4));
@@ -414,25 +413,27 @@ int vertical_slash_index(const void* q, const void* k, int Hq, int Hkv, int n, i
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int rc;
-  {
-    CUtensorMap tq, tk;
-    if (!make_tmap(&tq, q, (int64_t)Hq * n, d) || !make_tmap(&tk, k, (int64_t)Hkv * n, d)) return DSA_ERR_CUDA;
-    const dim3 gl((n + 127) / 128, Hkv * ((p.grp + 3) / 4));
-    if (d == 128) {
-      if ((rc = set_smem(vs_logits_kernel<128>, VSLogitLayout<128>::kSmemAlloc))) return rc;
-      vs_logits_kernel<128><<<gl, 256, VSLogitLayout<128>::kSmemAlloc, st>>>(tq, tk, p);
-    } else {
-      if ((rc = set_smem(vs_logits_kernel<64>, VSLogitLayout<64>::kSmemAlloc))) return rc;
-      vs_logits_kernel<64><<<gl, 256, VSLogitLayout<64>::kSmemAlloc, st>>>(tq, tk, p);
-    }
-    if ((rc = launch_check())) return rc;
+  CUtensorMap tq, tk;
+  if (!make_tmap(&tq, q, (int64_t)Hq * n, d) || !make_tmap(&tk, k, (int64_t)Hkv * n, d)) return DSA_ERR_CUDA;
+  const dim3 gl(ntiles, Hkv * ((p.grp + 3) / 4));
+  // pass 1 (row maxima and sums per key tile), the rows' log-sum-exp, pass 2
+  // (column sums and diagonal partials); the logits are computed in both passes
+  if (d == 128) {
+    if ((rc = set_smem(vs_score_kernel<128, 1>, VSScoreLayout<128>::kSmemAlloc)) ||
+        (rc = set_smem(vs_score_kernel<128, 2>, VSScoreLayout<128>::kSmemAlloc)))
+      return rc;
+    vs_score_kernel<128, 1><<<gl, 256, VSScoreLayout<128>::kSmemAlloc, st>>>(tq, tk, p);
+  } else {
+    if ((rc = set_smem(vs_score_kernel<64, 1>, VSScoreLayout<64>::kSmemAlloc)) ||
+        (rc = set_smem(vs_score_kernel<64, 2>, VSScoreLayout<64>::kSmemAlloc)))
+      return rc;
+    vs_score_kernel<64, 1><<<gl, 256, VSScoreLayout<64>::kSmemAlloc, st>>>(tq, tk, p);
   }
-  dim3 gt(ntiles, Hq);
-  vs_pass1_kernel<<<gt, 256, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
   vs_lse_kernel<<<Hq, 64, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
-  vs_pass2_kernel<<<gt, 256, 0, st>>>(p);
+  if (d == 128) vs_score_kernel<128, 2><<<gl, 256, VSScoreLayout<128>::kSmemAlloc, st>>>(tq, tk, p);
+  else vs_score_kernel<64, 2><<<gl, 256, VSScoreLayout<64>::kSmemAlloc, st>>>(tq, tk, p);
   if ((rc = launch_check())) return rc;
   vs_slash_kernel<<<dim3((n + 255) / 256, Hq), 256, 0, st>>>(p);
   if ((rc = launch_check())) return rc;

@@ -4,14 +4,16 @@
 // vertical lines as 1x64 column tiles).
 //
 // Rows i_r = n - 64 + r.  The logits z = q_i.k_j * scale (log2 domain) of
-// those rows against every key come from one tcgen05 kernel (a dense
-// product).  Pass 1 then computes each row's log-sum-exp over its causal keys;
-// pass 2 forms the probabilities P[r][j] = 2^(z - lse_r) and sums them per key
-// column (vert) and per diagonal offset o = i_r - j (slash).  Both passes tile
-// the keys in blocks of 64 per CTA (one q-head) and sum in a fixed order, so
-// the scores are deterministic run to run.  Then a top-k per head and the
-// per-query-block plan (aligned 64x64 blocks for slashes, column entries for
-// verticals).
+// those rows against every key are a dense product and run on tcgen05, tiled
+// 128 keys per CTA; they are computed twice and never stored.  The first pass
+// keeps each row's maximum and sum of 2^z over the tile's causal keys (a
+// partial per tile); the partials give each row's log-sum-exp; the second pass
+// forms the probabilities P[r][j] = 2^(z - lse_r) of the tile in shared memory
+// and sums them per key column (vert, complete per tile) and per diagonal
+// offset o = i_r - j (slash, a partial per tile, combined over the at most two
+// tiles an offset spans).  Every sum runs in a fixed order, so the scores are
+// deterministic run to run.  Then a top-k per head and the per-query-block
+// plan (aligned 64x64 blocks for slashes, column entries for verticals).
 #pragma once
 
 #include <cuda.h>
@@ -23,15 +25,17 @@
 
 namespace dsa {
 
+constexpr int kVSTile = 128;              // keys per CTA of the two score passes
+constexpr int kVSDiag = kVSTile + 63;     // diagonal offsets one tile touches (191)
+
 struct VSParams {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
-  float* zlog;        // [Hq][64][n] logits of the last 64 queries, log2 domain (scale*log2e folded in)
   uint32_t* status;
   float* part;        // [Hq][ntiles][64][2]  pass-1 (max, sum) per tile and row (log2 domain)
   float* lse2;        // [Hq][64]
   float* vert;        // [Hq][n]
-  float* slash_part;  // [Hq][ntiles][127]
+  float* slash_part;  // [Hq][ntiles][kVSDiag]
   float* slash;       // [Hq][n]
   int32_t* vsel;      // [Hq][n_vert]
   int32_t* ssel;      // [Hq][n_slash]
@@ -46,30 +50,37 @@ struct VSParams {
   float scale_log2;
 };
 
-// ---------------------------------------------------------------- logits on tensor cores
-// Z[h][r][j] = (q_{n-64+r} . k_j) * scale * log2(e) for the last 64 queries
-// of every q-head against all keys of its KV head: a dense product, so it runs
-// on tcgen05.  One CTA per (KV head, group of four q-heads, 128 keys): the
-// four heads' 64 rows form two M=128 tiles (TMA, 128-byte swizzle), the key
-// tile is N=128, fp32 accumulators in TMEM; 8 warps read the accumulators
-// back (one row per thread) and store the scaled row segment.  Causal masking
-// is left to the passes that read Z.
+// ---------------------------------------------------------------- the score passes
+// One CTA per (KV head, group of four q-heads, 128 keys): the four heads' last
+// 64 query rows form two M=128 tiles (TMA, 128-byte swizzle), the key tile is
+// N=128, the fp32 logits land in TMEM.  8 warps read them back, one row per
+// thread (warp w: tile w / 4, TMEM lane quarter w % 4).
+//   kPass = 1: each row's maximum and sum of 2^(z - max) over the tile's
+//              causal keys -> part;
+//   kPass = 2: P = 2^(z - lse) (0 past the causal boundary) of one tile at a
+//              time into shared memory (over the operand tiles, which the MMAs
+//              no longer need), then per key column the sum over the head's
+//              64 rows -> vert, and per diagonal offset the tile's partial sum
+//              -> slash_part.
 template <int D>
-struct VSLogitLayout {
+struct VSScoreLayout {
   static constexpr int NDH = D / 64;
   static constexpr int kHalf = 16384;        // one d-half of 128 rows x 128 B
   static constexpr int kTile = NDH * kHalf;
   static constexpr int kQA = 0, kQB = kTile, kK = 2 * kTile;
-  static constexpr int kBar = 3 * kTile;
+  static constexpr int kPStride = kVSTile + 1;                 // floats per row of P (padded)
+  static constexpr int kPBytes = 128 * kPStride * 4;           // one M=128 tile's P
+  static constexpr int kOperands = 3 * kTile;
+  static constexpr int kBar = (kOperands > kPBytes ? kOperands : kPBytes);
   static constexpr int kBytes = kBar + 64;
   static constexpr int kSmemAlloc = kBytes + 1024;
 };
 
-template <int D>
+template <int D, int kPass>
 __global__ void __launch_bounds__(256, 2)
-    vs_logits_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const VSParams p) {
-  using Lay = VSLogitLayout<D>;
+    vs_score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const VSParams p) {
+  using Lay = VSScoreLayout<D>;
   extern __shared__ uint8_t vs_smem_raw[];
   if (status_timed_out(p.status)) return;
   uint8_t* smem =
@@ -83,7 +94,7 @@ __global__ void __launch_bounds__(256, 2)
   const int g = blockIdx.y / nquads, quad = blockIdx.y % nquads;
   const int h0 = g * p.grp + 4 * quad;
   const int nh = min(4, p.grp - 4 * quad);
-  const int j0 = blockIdx.x * 128;
+  const int tileid = blockIdx.x, j0 = tileid * kVSTile;
   if (threadIdx.x == 0) {
     mbar_init(bar_full, 1);
     mbar_init(bar_mma, 1);
@@ -127,32 +138,91 @@ __global__ void __launch_bounds__(256, 2)
         }
       }
     }
-    umma_commit(bar_mma);
+    umma_commit(bar_mma);   // also once every operand read is done
   }
-  // epilogue: warp w reads TMEM lane quarter w%4 of tile w/4
   const int tile = warp >> 2, q4 = warp & 3;
   const int row = q4 * 32 + lane;
   const int hh = 2 * tile + (row >> 6), r = row & 63;
+  const int irow = p.n - 64 + r;               // this row's query position
+  const int h = h0 + min(hh, nh - 1);
   const bool ok = mbar_wait_warp(bar_mma, 0, ab);
-  if (ok && hh < nh) {
-    tc_fence_after();
-    float* dst = p.zlog + ((size_t)(h0 + hh) * 64 + r) * p.n + j0;
-    const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16) + 128u * (uint32_t)tile;
-    const int nchunk = min(128, p.n - j0) / 32;   // the last tile of an n % 128 == 64 sequence has 64 keys
+  const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16) + 128u * (uint32_t)tile;
+  if (kPass == 1) {
+    if (ok) {
+      tc_fence_after();
+      float m = -INFINITY, sum = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < kVSTile / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(ta + 32 * c, v);
+        tmem_wait_ld();
+        reg_fence(v);
+        float z[32];
+        float mc = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (c >= nchunk) break;
-      uint32_t v[32];
-      tmem_ld32(ta + 32 * c, v);
-      tmem_wait_ld();
-      reg_fence(v);
+        for (int x = 0; x < 32; ++x) {
+          z[x] = (j0 + 32 * c + x <= irow) ? __uint_as_float(v[x]) * p.scale_log2 : -INFINITY;
+          mc = fmaxf(mc, z[x]);
+        }
+        if (mc == -INFINITY) continue;
+        const float mn = fmaxf(m, mc);
+        float s = 0.f;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 w = make_float4(__uint_as_float(v[4 * q]) * p.scale_log2, __uint_as_float(v[4 * q + 1]) * p.scale_log2,
-                                     __uint_as_float(v[4 * q + 2]) * p.scale_log2,
-                                     __uint_as_float(v[4 * q + 3]) * p.scale_log2);
-        *reinterpret_cast<float4*>(dst + 32 * c + 4 * q) = w;
+        for (int x = 0; x < 32; ++x) s += ex2_approx(z[x] - mn);
+        sum = (m == -INFINITY ? 0.f : sum * ex2_approx(m - mn)) + s;
+        m = mn;
       }
+      if (hh < nh) {
+        float* o = p.part + (((size_t)h * p.ntiles + tileid) * 64 + r) * 2;
+        o[0] = m;
+        o[1] = sum;
+      }
+    }
+  } else {
+    // P of one M=128 tile at a time in shared memory (the operands are dead:
+    // every MMA, and so every operand read, completed before bar_mma)
+    float* P = reinterpret_cast<float*>(smem);
+    const float lse = p.lse2[(size_t)h * 64 + r];
+    fence_proxy_async_smem();   // the operands' async-proxy reads are ordered before these writes
+    for (int t2 = 0; t2 < 2; ++t2) {
+      if (tile == t2 && ok) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < kVSTile / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(ta + 32 * c, v);
+          tmem_wait_ld();
+          reg_fence(v);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const float z = __uint_as_float(v[x]) * p.scale_log2;
+            P[row * Lay::kPStride + 32 * c + x] = (j0 + 32 * c + x <= irow) ? ex2_approx(z - lse) : 0.f;
+          }
+        }
+      }
+      __syncthreads();
+      // the two heads of tile t2: key columns (256 sums) and diagonal partials
+      for (int x = threadIdx.x; x < 2 * kVSTile; x += 256) {
+        const int hx = x / kVSTile, c = x % kVSTile;
+        const int hq = 2 * t2 + hx;
+        if (hq < nh && j0 + c < p.n) {
+          float s = 0.f;
+          for (int rr = 0; rr < 64; ++rr) s += P[(hx * 64 + rr) * Lay::kPStride + c];
+          p.vert[(size_t)(h0 + hq) * p.n + j0 + c] = s;
+        }
+      }
+      for (int x = threadIdx.x; x < 2 * kVSDiag; x += 256) {
+        const int hx = x / kVSDiag, od = x % kVSDiag;
+        const int hq = 2 * t2 + hx;
+        if (hq < nh) {
+          // offset o = i_r - j = (n - 64 + r) - (j0 + c) = n - 64 - j0 - 127 + od, so c = r + 127 - od
+          const int rlo = max(0, od - (kVSTile - 1)), rhi = min(63, od);
+          float s = 0.f;
+          for (int rr = rlo; rr <= rhi; ++rr) s += P[(hx * 64 + rr) * Lay::kPStride + (rr + kVSTile - 1 - od)];
+          p.slash_part[((size_t)(h0 + hq) * p.ntiles + tileid) * kVSDiag + od] = s;
+        }
+      }
+      __syncthreads();
     }
   }
   tc_fence_before();
@@ -160,46 +230,6 @@ __global__ void __launch_bounds__(256, 2)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
-  }
-}
-
-// z[r][c] (log2 domain) of rows r of the last-64 queries of head h and keys
-// j0+c, c < 64, read from the logits above; -inf where j0 + c > i_r.
-__device__ __forceinline__ void vs_load_tile(const VSParams& p, int h, int tile, float* Z) {
-  const int j0 = tile * 64;
-  const int i0 = p.n - 64;
-  const float* src = p.zlog + (size_t)h * 64 * p.n + j0;
-  for (int x = threadIdx.x; x < 64 * 16; x += 256) {
-    const int r = x >> 4, c4 = (x & 15) * 4;
-    const float4 v = __ldg(reinterpret_cast<const float4*>(src + (size_t)r * p.n + c4));
-    Z[r * 65 + c4 + 0] = (j0 + c4 + 0 <= i0 + r) ? v.x : -INFINITY;
-    Z[r * 65 + c4 + 1] = (j0 + c4 + 1 <= i0 + r) ? v.y : -INFINITY;
-    Z[r * 65 + c4 + 2] = (j0 + c4 + 2 <= i0 + r) ? v.z : -INFINITY;
-    Z[r * 65 + c4 + 3] = (j0 + c4 + 3 <= i0 + r) ? v.w : -INFINITY;
-  }
-  __syncthreads();
-}
-
-// Pass 1: per (tile, head): row max and sum of exp2 over the tile's keys.
-__global__ void __launch_bounds__(256) vs_pass1_kernel(const VSParams p) {
-  __shared__ __align__(16) float Z[64 * 65];
-  const int tile = blockIdx.x, h = blockIdx.y;
-  vs_load_tile(p, h, tile, Z);
-  // 4 threads per row
-  const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
-  float mx = -INFINITY;
-  for (int c = q; c < 64; c += 4) mx = fmaxf(mx, Z[r * 65 + c]);
-  mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
-  float s = 0.f;
-  if (mx != -INFINITY)
-    for (int c = q; c < 64; c += 4) s += exp2f(Z[r * 65 + c] - mx);
-  s += __shfl_xor_sync(0xFFFFFFFFu, s, 1);
-  s += __shfl_xor_sync(0xFFFFFFFFu, s, 2);
-  if (q == 0) {
-    float* o = p.part + (((size_t)h * p.ntiles + tile) * 64 + r) * 2;
-    o[0] = mx;
-    o[1] = s;
   }
 }
 
@@ -217,45 +247,19 @@ __global__ void __launch_bounds__(64) vs_lse_kernel(const VSParams p) {
   p.lse2[h * 64 + r] = M + log2f(L);
 }
 
-// Pass 2: probabilities of the tile; column sums (complete) and diagonal
-// partial sums of the tile's 127 offsets.
-__global__ void __launch_bounds__(256) vs_pass2_kernel(const VSParams p) {
-  __shared__ __align__(16) float Z[64 * 65];
-  const int tile = blockIdx.x, h = blockIdx.y;
-  vs_load_tile(p, h, tile, Z);
-  for (int x = threadIdx.x; x < 64 * 64; x += 256) {
-    const int r = x >> 6, c = x & 63;
-    const float z = Z[r * 65 + c];
-    Z[r * 65 + c] = (z == -INFINITY) ? 0.f : exp2f(z - p.lse2[h * 64 + r]);
-  }
-  __syncthreads();
-  const int t = threadIdx.x;
-  if (t < 64) {
-    float s = 0.f;
-    for (int r = 0; r < 64; ++r) s += Z[r * 65 + t];
-    p.vert[(size_t)h * p.n + tile * 64 + t] = s;
-  } else if (t < 64 + 127) {
-    // offset index od: o = n - 127 - 64*tile + od ; key column c = r + 63 - od
-    const int od = t - 64;
-    float s = 0.f;
-    const int rlo = max(0, od - 63), rhi = min(63, od);
-    for (int r = rlo; r <= rhi; ++r) s += Z[r * 65 + (r + 63 - od)];
-    p.slash_part[((size_t)h * p.ntiles + tile) * 127 + od] = s;
-  }
-}
-
 // slash[o] = sum of the (at most two) tile partials covering offset o, in tile order.
 __global__ void __launch_bounds__(256) vs_slash_kernel(const VSParams p) {
   const int h = blockIdx.y;
   const int o = blockIdx.x * 256 + threadIdx.x;
   if (o >= p.n) return;
-  // tile t covers offsets [n - 127 - 64t, n - 1 - 64t]
-  const int tlo = max(0, (p.n - 127 - o + 63) >> 6);   // ceil((n-127-o)/64), clamped
-  const int thi = min(p.ntiles - 1, (p.n - 1 - o) >> 6);
+  // tile t covers offsets [n - 64 - kVSTile*t - (kVSTile - 1), n - 1 - kVSTile*t]
+  const int base = p.n - 64 - (kVSTile - 1);
+  const int tlo = max(0, (base - o + kVSTile - 1) / kVSTile);   // ceil((base - o) / kVSTile), clamped
+  const int thi = min(p.ntiles - 1, (p.n - 1 - o) / kVSTile);
   float s = 0.f;
   for (int t = tlo; t <= thi; ++t) {
-    const int od = o - (p.n - 127 - 64 * t);
-    if (od >= 0 && od < 127) s += p.slash_part[((size_t)h * p.ntiles + t) * 127 + od];
+    const int od = o - (base - kVSTile * t);
+    if (od >= 0 && od < kVSDiag) s += p.slash_part[((size_t)h * p.ntiles + t) * kVSDiag + od];
   }
   p.slash[(size_t)h * p.n + o] = s;
 }
