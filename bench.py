@@ -48,8 +48,8 @@ import synth  # noqa: E402
 # (dram__bytes_read.sum + dram__bytes_write.sum) of this bench's command, kept
 # with the kernel revision they were taken on (profiles/ holds the summary);
 # the line reports null for any other revision or workload.
-BSA_KERNEL_REVISION = "tile-skip-1"
-BSA_TRAFFIC = {}   # {(revision, workload): bytes}
+BSA_KERNEL_REVISION = "tile-skip-2"
+BSA_TRAFFIC = {("tile-skip-2", "llama3-8b-128k-bs10"): 1.69e9 + 1.02e9}   # {(revision, workload): bytes}
 UNIT = "TFLOP/s"
 DIAG_ELEMS = 64 * 65 // 2
 
@@ -180,11 +180,11 @@ def barrier(world: int):
 
 # ------------------------------------------------------------------ our arm
 
-def workload_config(workload: str, world: int) -> dict:
+def workload_config(workload: str, world: int, hq=None, hkv=None) -> dict:
     """The prefill workload's description, the same on both arms."""
     p = synth.CONFIGS[workload]
     kf, rho = p.get("k_fixed", 0), p.get("keep_ratio", 0.0)
-    return {"workload": workload, "Hq": p["Hq"], "Hkv": p["Hkv"], "seq_len": p["n"], "head_dim": p["d"],
+    return {"workload": workload, "Hq": hq or p["Hq"], "Hkv": hkv or p["Hkv"], "seq_len": p["n"], "head_dim": p["d"],
             "keep": f"k_fixed={kf}" if kf else f"ratio={rho}+sink+diag", "block": 64,
             "l2": "inputs larger than L2 (Q 1.07 GB, K/V 268 MB each at 128K), no flush",
             "parallelism": f"independent layer per GPU x{world}"}
@@ -196,7 +196,7 @@ def run_ours(args, rank, world, local):
     dsa.load_library()
     dev = torch.device("cuda", local)
     p = synth.CONFIGS[args.workload]
-    w = synth.make_prefill(args.workload, device=dev, seed=rank_seed(args.workload, rank))
+    w = synth.make_prefill(args.workload, device=dev, seed=rank_seed(args.workload, rank), Hq=args.hq, Hkv=args.hkv)
     Hq, n, d = w.q.shape
     kf, rho = p.get("k_fixed", 0), p.get("keep_ratio", 0.0)
     kcap = dsa.block_index_capacity(n, kf, rho)
@@ -292,7 +292,7 @@ def run_ours(args, rank, world, local):
         "metric": metric_name(args.workload), "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(args.workload, world), selected_block_density=round(density, 5)),
+        "config": dict(workload_config(args.workload, world, args.hq, args.hkv), selected_block_density=round(density, 5)),
         "breakdown_ms": {"index": round(index_ms, 4), "attention": round(attn_ms, 4)},
         "index_roofline": index_roof,
         "index_reuse": reuse,
@@ -790,6 +790,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-layers", action="store_true", help="skip the 32K and 1M layers")
+    ap.add_argument("--hq", type=int, default=None,
+                    help="query heads (default: the workload's; fewer for a reduced case to profile)")
+    ap.add_argument("--hkv", type=int, default=None, help="KV heads (default: the workload's)")
     ap.add_argument("--sustained-s", type=float, default=3.0,
                     help="seconds of back-to-back attention launches for the sustained-peak line (0: skip)")
     ap.add_argument("--decode-batch", type=int, default=16,

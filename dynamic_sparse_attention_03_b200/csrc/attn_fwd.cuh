@@ -251,10 +251,13 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per_qb = p.Hkv * p.nquads;
-  const int qb = p.nQB - 1 - (int)(blockIdx.x / per_qb);   // heaviest query blocks first
-  const int rem = (int)(blockIdx.x % per_qb);
-  const int g = rem / p.nquads, quad = rem % p.nquads;
+  // Work items run KV head by KV head, heaviest query blocks first within a
+  // head: the CTAs in flight together read one head's key/value blocks, which
+  // stay in L2 for all of them.
+  const int per_head = p.nQB * p.nquads;
+  const int g = (int)(blockIdx.x / per_head);
+  const int rem = (int)(blockIdx.x % per_head);
+  const int qb = p.nQB - 1 - rem / p.nquads, quad = rem % p.nquads;
   const int h0 = g * p.grp + 4 * quad;
   const int nh = min(4, p.grp - 4 * quad);
   const bool hasB = nh > 2;
@@ -315,13 +318,17 @@ __global__ void __launch_bounds__(384, 1)
     if (isK && lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
+      // the query tile is read once: its L2 lines go first, ahead of the
+      // key/value blocks other query blocks reuse
+      const uint64_t once = l2_policy_evict_first();
       mbar_arrive_expect_tx(bar(AB_Q), (uint32_t)(2 * Lay::kTile));
 #pragma unroll
       for (int hh = 0; hh < 4; ++hh) {
         const int h = h0 + min(hh, nh - 1);
 #pragma unroll
         for (int dh = 0; dh < Lay::NDH; ++dh)
-          tma_load_2d(sQ(hh >> 1) + dh * Lay::kHalf + (hh & 1) * 8192, &tmQ, dh * 64, h * p.n + qb * 64, bar(AB_Q));
+          tma_load_2d_hint(sQ(hh >> 1) + dh * Lay::kHalf + (hh & 1) * 8192, &tmQ, dh * 64, h * p.n + qb * 64,
+                           bar(AB_Q), once);
       }
     }
     if (!isK && lane == 0) prefetch_tmap(&tmV);
@@ -659,6 +666,7 @@ __global__ void __launch_bounds__(384, 1)
       const int i = qb * 64 + r;
       const float inv = (any && l_run > 0.f) ? 1.0f / l_run : 0.f;
       __nv_bfloat16* orow = p.o + ((size_t)h * p.n + i) * D;
+      const uint64_t once = l2_policy_evict_first();   // written once, not read here again
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -677,7 +685,7 @@ __global__ void __launch_bounds__(384, 1)
           w.y = pack_bf16x2(__uint_as_float(ov[q * 8 + 2]) * inv, __uint_as_float(ov[q * 8 + 3]) * inv);
           w.z = pack_bf16x2(__uint_as_float(ov[q * 8 + 4]) * inv, __uint_as_float(ov[q * 8 + 5]) * inv);
           w.w = pack_bf16x2(__uint_as_float(ov[q * 8 + 6]) * inv, __uint_as_float(ov[q * 8 + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = w;
+          st_global_v4_evict_first(orow + c * 32 + q * 8, w, once);
         }
       }
       if (p.lse) {
