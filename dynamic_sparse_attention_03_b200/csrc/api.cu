@@ -96,6 +96,20 @@ bool make_tmap_f16(CUtensorMap* m, const void* base, int64_t rows, int d, int bo
   return r == CUDA_SUCCESS;
 }
 
+// 2D bf16 view [rows][d] with a 64-element (128-byte) x box_rows box and 128-byte swizzle.
+bool make_tmap_rows(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool validate_env() {
   const char* v = std::getenv("DSA_VALIDATE");
   return v && v[0] == '1';
@@ -580,12 +594,15 @@ int kmeans_clusters(const void* k_cache, int B, int Hkv, int S, int d, int n_ctx
   if (C > n_ctx) return DSA_ERR_INVALID_ARG;   // every starting segment holds a key
   if ((d != 64 && d != 128) || C > kKmMaxC) return DSA_ERR_UNSUPPORTED;
   if ((int64_t)B * Hkv > 65535 || (int64_t)S * d >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hkv * S >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(k_cache) || !aligned16(centroids)) return DSA_ERR_INVALID_ARG;
   const int BG = B * Hkv;
   WsCarve c(ws);
   uint32_t* status = static_cast<uint32_t*>(c.take(kStatusBytes));
-  (void)status;
   float* cnorm = static_cast<float*>(c.take((size_t)BG * C * 4));
+  // the centroids as bf16 hi / lo halves, the assignment's tensor-core operands
+  auto* chi = static_cast<__nv_bfloat16*>(c.take((size_t)BG * C * d * 2));
+  auto* clo = static_cast<__nv_bfloat16*>(c.take((size_t)BG * C * d * 2));
   if (!ws) {
     *ws_bytes = c.off;
     return DSA_OK;
@@ -596,25 +613,33 @@ int kmeans_clusters(const void* k_cache, int B, int Hkv, int S, int d, int n_ctx
   p.k = static_cast<const __nv_bfloat16*>(k_cache);
   p.cent = centroids;
   p.cnorm = cnorm;
+  p.chi = chi;
+  p.clo = clo;
   p.assign = assign;
   p.off = offsets;
   p.tok = tokens;
+  p.status = status;
   p.S = S;
   p.n_ctx = n_ctx;
   p.C = C;
+  p.BG = BG;
+  CUtensorMap tk, th, tl;
+  if (!make_tmap_rows(&tk, k_cache, (int64_t)BG * S, d, 128) || !make_tmap_rows(&th, chi, (int64_t)BG * C, d, 128) ||
+      !make_tmap_rows(&tl, clo, (int64_t)BG * C, d, 128))
+    return DSA_ERR_CUDA;
   int rc;
-  const dim3 gi(C, BG), ga((n_ctx + 127) / 128, BG), gu((C + 7) / 8, BG);
+  const dim3 gi(C, BG), ga((n_ctx + 255) / 256, BG), gu((C + 7) / 8, BG);
   if (d == 128) {
-    if ((rc = set_smem(kmeans_assign_kernel<128>, KmAssignLayout<128>::kBytes))) return rc;
+    if ((rc = set_smem(kmeans_assign_kernel<128>, KmAssignLayout<128>::kSmemAlloc))) return rc;
     kmeans_init_kernel<128><<<gi, 128, 0, st>>>(p);
   } else {
-    if ((rc = set_smem(kmeans_assign_kernel<64>, KmAssignLayout<64>::kBytes))) return rc;
+    if ((rc = set_smem(kmeans_assign_kernel<64>, KmAssignLayout<64>::kSmemAlloc))) return rc;
     kmeans_init_kernel<64><<<gi, 64, 0, st>>>(p);
   }
   if ((rc = launch_check())) return rc;
   for (int it = 0; it < iters; ++it) {
-    if (d == 128) kmeans_assign_kernel<128><<<ga, 256, KmAssignLayout<128>::kBytes, st>>>(p);
-    else kmeans_assign_kernel<64><<<ga, 256, KmAssignLayout<64>::kBytes, st>>>(p);
+    if (d == 128) kmeans_assign_kernel<128><<<ga, 320, KmAssignLayout<128>::kSmemAlloc, st>>>(tk, th, tl, p);
+    else kmeans_assign_kernel<64><<<ga, 320, KmAssignLayout<64>::kSmemAlloc, st>>>(tk, th, tl, p);
     if ((rc = launch_check())) return rc;
     kmeans_csr_kernel<<<BG, 1024, 0, st>>>(p);
     if ((rc = launch_check())) return rc;

@@ -8,9 +8,11 @@
 //  kmeans_init_kernel:   centroid c = mean of the contiguous segment
 //                        [floor(c n / C), floor((c+1) n / C)) of the keys.
 //  kmeans_assign_kernel: every key to its nearest centroid (squared Euclidean
-//                        distance, ties to the lower cluster): a tiled fp32
-//                        key x centroid product (128 keys x 64 centroids per
-//                        step) with a running argmin of |c|^2 - 2 k.c.
+//                        distance, ties to the lower cluster): the key x
+//                        centroid product on tcgen05 (256 keys per CTA, the
+//                        centroids streamed 128 at a time as bf16 hi + lo
+//                        halves, two products) with a running argmin of
+//                        |c|^2 - 2 k.c per key.
 //  kmeans_csr_kernel:    cluster -> key map: counts, offsets and the keys of
 //                        each cluster in ascending token order (a stable
 //                        counting sort).
@@ -51,11 +53,22 @@ struct KmParams {
   const __nv_bfloat16* k;   // [BG][S][D]
   float* cent;              // [BG][C][D]
   float* cnorm;             // [BG][C] |c|^2
+  __nv_bfloat16* chi;       // [BG][C][D] bf16(c)          (the assignment's tensor-core operands)
+  __nv_bfloat16* clo;       // [BG][C][D] bf16(c - bf16(c))
   int32_t* assign;          // [BG][n_ctx]
   int32_t* off;             // [BG][C + 1]
   int32_t* tok;             // [BG][n_ctx]
-  int S, n_ctx, C;
+  uint32_t* status;
+  int S, n_ctx, C, BG;
 };
+
+// The assignment's operands for centroid value c: hi = bf16(c), lo =
+// bf16(c - hi).  Keys are bf16 exactly, so k.c = k.hi + k.lo to about 2^-17
+// of |k||c| (the two products accumulate in fp32).
+__device__ __forceinline__ void km_split(float c, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(c);
+  lo = __float2bfloat16_rn(c - __bfloat162float(hi));
+}
 
 // ---------------------------------------------------------------- init
 // One CTA of D threads per (cluster, batch x KV head): thread = dimension.
@@ -69,6 +82,7 @@ __global__ void __launch_bounds__(D) kmeans_init_kernel(const KmParams p) {
   for (int r = lo; r < hi; ++r, kr += D) s += __bfloat162float(*kr);
   const float mean = s / (float)(hi - lo);
   p.cent[((size_t)bg * p.C + c) * D + t] = mean;
+  km_split(mean, p.chi[((size_t)bg * p.C + c) * D + t], p.clo[((size_t)bg * p.C + c) * D + t]);
   float sq = mean * mean;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xFFFFFFFFu, sq, o);
@@ -83,114 +97,189 @@ __global__ void __launch_bounds__(D) kmeans_init_kernel(const KmParams p) {
 }
 
 // ---------------------------------------------------------------- assign
-// One CTA of 256 threads per (128 keys, batch x KV head).  Shared memory
-// holds the key tile transposed ([D][128] fp32) and a centroid chunk
-// transposed ([D][64]); thread (ty, tx) = (tid / 16, tid % 16) owns keys
-// 8 ty .. 8 ty + 7 and centroids 4 tx .. 4 tx + 3 of the chunk.
+// One CTA per (256 keys, batch x KV head).  Warp 0 loads the two 128-key
+// tiles once and streams the centroids through a 2-stage ring (TMA, 128-byte
+// swizzle: 128 centroids x D as bf16 hi and lo, and their |c|^2); warp 1
+// issues S_t = K_t C_hi^T + K_t C_lo^T (M = 128 keys, N = 128 centroids, fp32 in
+// TMEM, two buffers per key tile); warps 2-9 each own 32 keys (key tile t =
+// (w - 2) / 4, TMEM lane quarter w % 4) and keep a running argmin of
+// |c|^2 - 2 k.c over the chunks, which arrive in increasing centroid order (so
+// ties go to the lower cluster).  Every wait is bounded.
 template <int D>
 struct KmAssignLayout {
-  static constexpr int kKeys = 0;
-  static constexpr int kCent = D * 128 * 4;
-  static constexpr int kBytes = kCent + D * 64 * 4;
+  static constexpr int NDH = D / 64;
+  static constexpr int kHalf = 16384;                // 128 rows x 128 B
+  static constexpr int kTile = NDH * kHalf;          // 128 rows x D bf16
+  static constexpr int kK = 0;                       // two key tiles
+  static constexpr int kRing = 2 * kTile;            // [stage]: hi tile, lo tile
+  static constexpr int kStage = 2 * kTile;
+  static constexpr int kCn = kRing + 2 * kStage;     // [stage][128] |c|^2
+  static constexpr int kBar = kCn + 2 * 128 * 4;
+  static constexpr int kBytes = kBar + 128;
+  static constexpr int kSmemAlloc = kBytes + 1024;
 };
 
 template <int D>
-__global__ void __launch_bounds__(256) kmeans_assign_kernel(const KmParams p) {
+__global__ void __launch_bounds__(320, 1)
+    kmeans_assign_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmH,
+                         const __grid_constant__ CUtensorMap tmL, const KmParams p) {
   using Lay = KmAssignLayout<D>;
-  extern __shared__ __align__(16) uint8_t kas[];
-  float* ks = reinterpret_cast<float*>(kas + Lay::kKeys);   // [D][128]
-  float* cs = reinterpret_cast<float*>(kas + Lay::kCent);   // [D][64]
-  const int bg = blockIdx.y, t0 = blockIdx.x * 128;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  // key tile, transposed (rows past n_ctx are zero and never written back)
-  for (int x = tid; x < 128 * D / 8; x += 256) {
-    const int row = x / (D / 8), c8 = x % (D / 8);
-    float f[8];
-    if (t0 + row < p.n_ctx) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.k + ((size_t)bg * p.S + t0 + row) * D) + c8);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  extern __shared__ uint8_t km_smem_raw[];
+  if (status_timed_out(p.status)) return;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(km_smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t bar0 = sb + Lay::kBar;
+  const uint32_t kbar = bar0;                                    // key tiles landed
+  auto full = [&](int s) { return bar0 + 8u * (1 + s); };        // centroid stage landed (+ |c|^2 stored)
+  auto empty = [&](int s) { return bar0 + 8u * (3 + s); };       // stage read by the MMAs
+  auto sfull = [&](int b) { return bar0 + 8u * (5 + b); };       // S buffer b computed (both key tiles)
+  auto sempty = [&](int b) { return bar0 + 8u * (7 + b); };      // S buffer b read by the epilogue
+  const uint32_t done = bar0 + 8u * 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kBar + 80);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kBar + 84);
+  float* cn_s = reinterpret_cast<float*>(smem + Lay::kCn);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bg = blockIdx.y, t0 = blockIdx.x * 256;
+  const int nchunks = (p.C + 127) / 128;
+  if (threadIdx.x == 0) {
+    mbar_init(kbar, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(full(s), 2);   // the TMA bytes' arrival + the |c|^2 stores' arrival
+      mbar_init(empty(s), 1);
+      mbar_init(sfull(s), 1);
+      mbar_init(sempty(s), 8);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const AbortState ab{abort_flag, p.status};
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      mbar_arrive_expect_tx(kbar, (uint32_t)(2 * Lay::kTile));
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const float2 v = __bfloat1622float2(h2[a]);
-        f[2 * a] = v.x;
-        f[2 * a + 1] = v.y;
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int dh = 0; dh < Lay::NDH; ++dh)
+          tma_load_2d(sb + Lay::kK + t * Lay::kTile + dh * Lay::kHalf, &tmK, dh * 64, bg * p.S + t0 + 128 * t, kbar);
+    }
+    int c = 0;
+    for (; c < nchunks; ++c) {
+      const int s = c & 1;
+      if (c >= 2 && !mbar_wait_warp(empty(s), ((c >> 1) - 1) & 1, ab)) break;
+      const int c0 = c * 128;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(full(s), (uint32_t)(2 * Lay::kTile));
+#pragma unroll
+        for (int dh = 0; dh < Lay::NDH; ++dh) {
+          tma_load_2d(sb + Lay::kRing + s * Lay::kStage + dh * Lay::kHalf, &tmH, dh * 64, bg * p.C + c0, full(s));
+          tma_load_2d(sb + Lay::kRing + s * Lay::kStage + Lay::kTile + dh * Lay::kHalf, &tmL, dh * 64,
+                      bg * p.C + c0, full(s));
+        }
       }
-    } else {
-#pragma unroll
-      for (int a = 0; a < 8; ++a) f[a] = 0.f;
+      // |c|^2 of the chunk (+inf past the last centroid: never the argmin),
+      // once the epilogue has read this slot's values of chunk c - 2
+      if (c >= 2 && !mbar_wait_warp(sempty(s), ((c >> 1) - 1) & 1, ab)) break;
+      for (int x = lane; x < 128; x += 32)
+        cn_s[s * 128 + x] = (c0 + x < p.C) ? p.cnorm[(size_t)bg * p.C + c0 + x] : __int_as_float(0x7f800000);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full(s));
     }
-#pragma unroll
-    for (int a = 0; a < 8; ++a) ks[(c8 * 8 + a) * 128 + row] = f[a];
-  }
-  float best[8];
-  int bidx[8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    best[r] = __int_as_float(0x7f800000);
-    bidx[r] = 0;
-  }
-  const float* cent = p.cent + (size_t)bg * p.C * D;
-  const float* cn = p.cnorm + (size_t)bg * p.C;
-  for (int c0 = 0; c0 < p.C; c0 += 64) {
-    __syncthreads();
-    for (int x = tid; x < 64 * D / 4; x += 256) {
-      const int cc = x / (D / 4), d4 = x % (D / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c0 + cc < p.C) v = __ldg(reinterpret_cast<const float4*>(cent + (size_t)(c0 + cc) * D) + d4);
-      cs[(d4 * 4 + 0) * 64 + cc] = v.x;
-      cs[(d4 * 4 + 1) * 64 + cc] = v.y;
-      cs[(d4 * 4 + 2) * 64 + cc] = v.z;
-      cs[(d4 * 4 + 3) * 64 + cc] = v.w;
+    // this warp's copies in flight land before the CTA exits
+    if (lane == 0) {
+      mbar_wait_cleanup(kbar, 0, 200000000ull);
+      for (int u = max(0, c - 2); u < c; ++u) mbar_wait_cleanup(full(u & 1), (u >> 1) & 1, 200000000ull);
     }
-    __syncthreads();
-    float acc[8][4];
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (warp-uniform walk)
+    const bool issuer = elect_one();
+    const uint32_t idesc = umma_idesc_bf16(128, 128, 0);
+    bool ok = mbar_wait_warp(kbar, 0, ab);
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int s = c & 1, b = c & 1;
+      if (!(ok = mbar_wait_warp(full(s), (c >> 1) & 1, ab))) break;
+      if (c >= 2 && !(ok = mbar_wait_warp(sempty(b), ((c >> 1) - 1) & 1, ab))) break;
+      tc_fence_after();
+      const uint32_t st = sb + Lay::kRing + s * Lay::kStage;
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
+      for (int t = 0; t < 2; ++t) {
+        const uint32_t dS = tmem + 256u * (uint32_t)t + 128u * (uint32_t)b;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[r][j] = 0.f;
-#pragma unroll 4
-    for (int dd = 0; dd < D; ++dd) {
-      const float4 ka = *reinterpret_cast<const float4*>(ks + dd * 128 + ty * 8);
-      const float4 kb = *reinterpret_cast<const float4*>(ks + dd * 128 + ty * 8 + 4);
-      const float4 cv = *reinterpret_cast<const float4*>(cs + dd * 64 + tx * 4);
-      const float kv[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
-      const float cc4[4] = {cv.x, cv.y, cv.z, cv.w};
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[r][j] = fmaf(kv[r], cc4[j], acc[r][j]);
-    }
-    // distance up to the key's own |k|^2: |c|^2 - 2 k.c; ties to the lower cluster
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + tx * 4 + j;
-      if (c < p.C) {
-        const float n2 = __ldg(cn + c);
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const float dist = fmaf(-2.f, acc[r][j], n2);
-          if (dist < best[r]) {   // clusters arrive in increasing order per thread
-            best[r] = dist;
-            bidx[r] = c;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)((kk >> 2) * Lay::kHalf + (kk & 3) * 32);
+          const uint64_t a = umma_desc_sw128(sb + Lay::kK + t * Lay::kTile + off, 16, 1024);
+          const uint64_t bh = umma_desc_sw128(st + off, 16, 1024);
+          const uint64_t bl = umma_desc_sw128(st + Lay::kTile + off, 16, 1024);
+          if (issuer) {
+            umma_bf16_ss(dS, a, bh, idesc, kk > 0 ? 1u : 0u);
+            umma_bf16_ss(dS, a, bl, idesc, 1u);
           }
         }
       }
-    }
-  }
-  // reduce over the 16 threads that share a key row (lanes tx = 0..15 of a half warp)
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) {
-      const float ob = __shfl_xor_sync(0xFFFFFFFFu, best[r], o);
-      const int oi = __shfl_xor_sync(0xFFFFFFFFu, bidx[r], o);
-      if (ob < best[r] || (ob == best[r] && oi < bidx[r])) {
-        best[r] = ob;
-        bidx[r] = oi;
+      if (issuer) {
+        umma_commit(empty(s));
+        umma_commit(sfull(b));
       }
+      __syncwarp();
     }
-    const int t = t0 + ty * 8 + r;
-    if (tx == 0 && t < p.n_ctx) p.assign[(size_t)bg * p.n_ctx + t] = bidx[r];
+    if (issuer) {
+      umma_commit(done);
+      mbar_wait_cleanup(done, 0, 200000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ argmin, one key per thread
+    const int t = (warp - 2) >> 2, q4 = warp & 3;
+    const int key = t0 + 128 * t + q4 * 32 + lane;
+    const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16) + 256u * (uint32_t)t;
+    float best = __int_as_float(0x7f800000);
+    int bidx = 0;
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      const int b = c & 1;
+      if (!(ok = mbar_wait_warp(sfull(b), (c >> 1) & 1, ab))) break;
+      // the |c|^2 stores are acquired from the producer's own arrival (the
+      // slot cannot move on to chunk c + 2 before this warp releases chunk c)
+      if (!(ok = mbar_wait_warp(full(c & 1), (c >> 1) & 1, ab))) break;
+      tc_fence_after();
+      const float* cn = cn_s + (c & 1) * 128;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t v[32];
+        tmem_ld32(ta + 128u * (uint32_t)b + 32u * (uint32_t)q, v);
+        tmem_wait_ld();
+        reg_fence(v);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const float dist = fmaf(-2.f, __uint_as_float(v[x]), cn[32 * q + x]);
+          if (dist < best) {   // centroids in increasing order: ties keep the lower one
+            best = dist;
+            bidx = c * 128 + 32 * q + x;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sempty(b));
+    }
+    if (ok && key < p.n_ctx) p.assign[(size_t)bg * p.n_ctx + key] = bidx;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -298,10 +387,12 @@ __global__ void __launch_bounds__(256) kmeans_update_kernel(const KmParams p) {
   const float inv = 1.f / (float)(b - a);
   float sq = 0.f;
   float* out = p.cent + ((size_t)bg * p.C + c) * D + lane * PER;
+  const size_t o2 = ((size_t)bg * p.C + c) * D + lane * PER;
 #pragma unroll
   for (int x = 0; x < PER; ++x) {
     const float m = s[x] * inv;
     out[x] = m;
+    km_split(m, p.chi[o2 + x], p.clo[o2 + x]);
     sq = fmaf(m, m, sq);
   }
 #pragma unroll
