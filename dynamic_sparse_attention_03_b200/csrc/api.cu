@@ -208,8 +208,10 @@ int launch_decode(const DecodeParams& p, int B, int Hkv, int nchmax, size_t sel_
   int rc;
   decode_score_kernel<D, G><<<dim3(B * Hkv, (p.nb + 63) / 64), 256, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
-  if ((rc = set_smem(decode_select_kernel<D, G, 256>, sel_smem))) return rc;
-  decode_select_kernel<D, G, 256><<<B * Hkv, 256, sel_smem, st>>>(p);
+  if ((rc = set_smem(decode_topk_kernel<256>, sel_smem))) return rc;
+  decode_topk_kernel<256><<<B * Hkv * G, 256, sel_smem, st>>>(p);
+  if ((rc = launch_check())) return rc;
+  decode_union_kernel<G, 256><<<B * Hkv, 256, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
   if ((rc = set_smem(decode_attn_kernel<D, G>, DecLayout<D>::kBytes))) return rc;
   decode_attn_kernel<D, G><<<dim3(B * Hkv, nchmax), kDecThreads, DecLayout<D>::kBytes, st>>>(p);
@@ -226,8 +228,12 @@ int launch_cluster_decode(const ClusterParams& cp, int B, int Hkv, int nchmax, s
   sp.scores = const_cast<float*>(cp.scores);
   decode_score_kernel<D, G><<<dim3(B * Hkv, (cp.C + 63) / 64), 256, 0, st>>>(sp);
   if ((rc = launch_check())) return rc;
-  if ((rc = set_smem(cluster_select_kernel<D, G, 256>, sel_smem))) return rc;
-  cluster_select_kernel<D, G, 256><<<B * Hkv, 256, sel_smem, st>>>(cp);
+  if ((rc = set_smem(cluster_topk_kernel<256>, sel_smem))) return rc;
+  cluster_topk_kernel<256><<<B * Hkv * G, 256, sel_smem, st>>>(cp);
+  if ((rc = launch_check())) return rc;
+  const size_t uni_smem = (size_t)(cp.C + 1) * 4 + (size_t)cp.C * 5;
+  if ((rc = set_smem(cluster_union_kernel<G, 256>, uni_smem))) return rc;
+  cluster_union_kernel<G, 256><<<B * Hkv, 256, uni_smem, st>>>(cp);
   if ((rc = launch_check())) return rc;
   if (cp.dp.n_packed > 0) {
     if ((rc = set_smem(cluster_stream_attn_kernel<D, G>, ClStreamLayout<D>::kBytes))) return rc;
@@ -532,12 +538,13 @@ int sparse_decode_attn(const void* q, const void* k_cache, const void* v_cache, 
   const int ncand = force_last ? nb - 1 : nb;
   const int count = std::min(keep, ncand) + force_last;
   if (sel_idx && kcap < count) return DSA_ERR_CAPACITY;
-  const size_t sel_smem = (size_t)grp * nb * 4 + (size_t)nb * 4 + nb;
+  const size_t sel_smem = (size_t)nb * 8 + (size_t)((nb + 31) / 32) * 4;   // one q-head's scores, ids, bitmap
   if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
   const int nchmax = (nb + kDecChunk - 1) / kDecChunk;
   WsCarve c(ws);
   DecodeParams p{};
   p.status = static_cast<uint32_t*>(c.take(kStatusBytes));
+  p.kbits = static_cast<uint32_t*>(c.take((size_t)B * Hq * ((nb + 31) / 32) * 4));
   p.uidx = static_cast<int32_t*>(c.take((size_t)B * Hkv * nb * 4));
   p.umask = static_cast<uint8_t*>(c.take((size_t)B * Hkv * nb));
   p.ucnt = static_cast<int32_t*>(c.take((size_t)B * Hkv * 4));
@@ -687,13 +694,15 @@ int cluster_decode_attn(const void* q, const void* k_cache, const void* v_cache,
   if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(centroids)) return DSA_ERR_INVALID_ARG;
   if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
   if (sel_idx && kcap < std::min(keep, C)) return DSA_ERR_CAPACITY;
-  const size_t sel_smem = (size_t)grp * C * 4 + (size_t)C * 12 + (size_t)(C + 1) * 4 + C;
+  // one q-head's candidate scores, ids, top ids, the offsets and a bitmap
+  const size_t sel_smem = (size_t)C * 12 + (size_t)(C + 1) * 4 + (size_t)((C + 31) / 32) * 4;
   if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
   const int nchmax = (S + kClChunk - 1) / kClChunk;
   WsCarve c(ws);
   ClusterParams cp{};
   DecodeParams& p = cp.dp;
   p.status = static_cast<uint32_t*>(c.take(kStatusBytes));
+  p.kbits = static_cast<uint32_t*>(c.take((size_t)B * Hq * ((C + 31) / 32) * 4));
   // union lists per (batch, KV head), rows padded to 16 entries (the head
   // masks are bulk-copied 16-byte aligned)
   const int lstride = (S + 15) & ~15;

@@ -22,13 +22,14 @@
 // Lloyd rounds run (assign, csr, update) `iters` times.
 //
 // Online decode:
-//  cluster_select_kernel: per (batch, KV head): the scores of the non-empty
-//                        clusters (q.c for every cluster comes from
-//                        decode_score_kernel, many CTAs), the top `keep` per head
-//                        (ties to the lower cluster), and the union of the
-//                        group's kept clusters flattened into one token list
-//                        with a per-token head mask, followed by the
-//                        unclustered tail [n_ctx, S) that every head attends.
+//  cluster_topk_kernel:  per (batch, q-head): the top `keep` non-empty
+//                        clusters by q.c (computed for every cluster by
+//                        decode_score_kernel, many CTAs), ties to the lower
+//                        cluster, as a bitmap;
+//  cluster_union_kernel: per (batch, KV head): the union of the group's kept
+//                        clusters flattened into one token list with a
+//                        per-token head mask, followed by the unclustered
+//                        tail [n_ctx, S) that every head attends.
 //  cluster_attn_kernel:  kClChunk entries of the union list per CTA: K and V rows
 //                        read by position from the cluster-ordered copy
 //                        (cluster_pack_kernel) when there is one, else
@@ -410,60 +411,85 @@ struct ClusterParams {
   int C, n_ctx;
 };
 
-template <int D, int GRP, int NT>
-__global__ void __launch_bounds__(NT) cluster_select_kernel(const ClusterParams cp) {
+// Two launches, so the top-k of every q-head runs in parallel: one CTA per
+// (batch, q-head) ranks the (batch, KV head)'s non-empty clusters by that
+// head's scores, keeps `keep` of them (ties to the lower cluster) and writes
+// them as a bitmap over cluster ids (and the optional selection outputs); one
+// CTA per (batch, KV head) ORs the group's bitmaps and flattens the kept
+// clusters into one token list with a per-token head mask (clusters in id
+// order, each cluster's tokens as the cluster -> key map lists them), then the
+// unclustered tail [n_ctx, S) that every head attends.
+template <int NT>
+__global__ void __launch_bounds__(NT) cluster_topk_kernel(const ClusterParams cp) {
   extern __shared__ __align__(16) uint8_t csm[];
   __shared__ SelectSmem sm;
   const DecodeParams& p = cp.dp;
-  const int bg = blockIdx.x;
-  const int b = bg / p.Hkv, g = bg % p.Hkv;
-  const int C = cp.C;
-  float* sc = reinterpret_cast<float*>(csm);                        // [GRP][C] (compacted candidates)
-  int32_t* cand = reinterpret_cast<int32_t*>(sc + (size_t)GRP * C);  // [C] non-empty cluster ids
-  int32_t* tmp = cand + C;                                           // [C]
-  int32_t* ubase = tmp + C;                                          // [C] union token offsets
-  int32_t* off = ubase + C;                                          // [C + 1] the cluster -> key offsets
-  uint8_t* mask = reinterpret_cast<uint8_t*>(off + C + 1);           // [C]
-  // the offsets come in once, coalesced: the union loop below reads them per
-  // cluster, which from global memory was a chain of dependent loads per warp
+  const int bh = blockIdx.x;   // b * Hq + h
+  const int b = bh / p.Hq, h = bh % p.Hq, g = h / p.grp;
+  const int bg = b * p.Hkv + g;
+  const int C = cp.C, nw = (C + 31) >> 5;
+  float* sc = reinterpret_cast<float*>(csm);                    // [C] candidates' scores
+  int32_t* cand = reinterpret_cast<int32_t*>(sc + C);           // [C] non-empty cluster ids
+  int32_t* tmp = cand + C;                                      // [C]
+  int32_t* off = tmp + C;                                       // [C + 1]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(off + C + 1);    // [nw]
   const int32_t* goff = cp.off + (size_t)bg * (C + 1);
   for (int x = threadIdx.x; x <= C; x += NT) off[x] = goff[x];
+  for (int x = threadIdx.x; x < nw; x += NT) bits[x] = 0u;
   __syncthreads();
   // non-empty clusters, ascending (block scan over per-thread ranges)
   const int per = (C + NT - 1) / NT;
   const int c0 = min(C, (int)threadIdx.x * per), c1 = min(C, c0 + per);
   int ne = 0;
-  for (int c = c0; c < c1; ++c) {
-    mask[c] = 0;
-    ne += off[c + 1] > off[c];
-  }
+  for (int c = c0; c < c1; ++c) ne += off[c + 1] > off[c];
   int ncand;
   int pos = block_excl_scan<NT>(ne, sm, ncand);
   for (int c = c0; c < c1; ++c)
     if (off[c + 1] > off[c]) cand[pos++] = c;
   __syncthreads();
-  // the candidates' scores, computed for every cluster by decode_score_kernel
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* gsc = cp.scores + ((size_t)b * p.Hq + g * GRP) * C;   // the group's rows are contiguous
-  for (int x = threadIdx.x; x < GRP * ncand; x += NT) {
-    const int hh = x / ncand, y = x % ncand;
-    sc[(size_t)hh * C + y] = gsc[(size_t)hh * C + cand[y]];
-  }
+  const float* gsc = cp.scores + (size_t)bh * C;
+  for (int y = threadIdx.x; y < ncand; y += NT) sc[y] = gsc[cand[y]];
   __syncthreads();
   const int e = min(p.keep, ncand);
-  for (int hh = 0; hh < GRP; ++hh) {
-    const int cnt = topk_ascending<NT>(sc + (size_t)hh * C, ncand, e, 0, ncand, tmp, C, sm);
-    __syncthreads();
-    const int h = g * GRP + hh;
-    for (int x = threadIdx.x; x < cnt; x += NT) mask[cand[tmp[x]]] |= (uint8_t)(1u << hh);
-    if (p.sel_idx) {
-      int32_t* out = p.sel_idx + ((size_t)b * p.Hq + h) * p.kcap;
-      for (int x = threadIdx.x; x < p.kcap; x += NT) out[x] = x < cnt ? cand[tmp[x]] : -1;
-    }
-    if (p.sel_cnt && threadIdx.x == 0) p.sel_cnt[(size_t)b * p.Hq + h] = cnt;
-    __syncthreads();
+  const int cnt = topk_ascending<NT>(sc, ncand, e, 0, ncand, tmp, C, sm);
+  __syncthreads();
+  for (int x = threadIdx.x; x < cnt; x += NT) {
+    const int c = cand[tmp[x]];
+    atomicOr(&bits[c >> 5], 1u << (c & 31));
   }
-  // the union's tokens in cluster order, then the tail
+  if (p.sel_idx) {
+    int32_t* out = p.sel_idx + (size_t)bh * p.kcap;
+    for (int x = threadIdx.x; x < p.kcap; x += NT) out[x] = x < cnt ? cand[tmp[x]] : -1;
+  }
+  if (p.sel_cnt && threadIdx.x == 0) p.sel_cnt[bh] = cnt;
+  __syncthreads();
+  uint32_t* gb = p.kbits + (size_t)bh * nw;
+  for (int x = threadIdx.x; x < nw; x += NT) gb[x] = bits[x];
+}
+
+template <int GRP, int NT>
+__global__ void __launch_bounds__(NT) cluster_union_kernel(const ClusterParams cp) {
+  extern __shared__ __align__(16) uint8_t csm[];
+  __shared__ SelectSmem sm;
+  const DecodeParams& p = cp.dp;
+  const int bg = blockIdx.x;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int C = cp.C, nw = (C + 31) >> 5;
+  int32_t* off = reinterpret_cast<int32_t*>(csm);   // [C + 1] the cluster -> key offsets
+  int32_t* ubase = off + C + 1;                     // [C] union token offsets
+  uint8_t* mask = reinterpret_cast<uint8_t*>(ubase + C);   // [C]
+  const int32_t* goff = cp.off + (size_t)bg * (C + 1);
+  for (int x = threadIdx.x; x <= C; x += NT) off[x] = goff[x];
+  const uint32_t* gb = p.kbits + ((size_t)b * p.Hq + g * GRP) * nw;   // the group's rows are contiguous
+  for (int c = threadIdx.x; c < C; c += NT) {
+    uint32_t m = 0u;
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) m |= ((gb[(size_t)hh * nw + (c >> 5)] >> (c & 31)) & 1u) << hh;
+    mask[c] = (uint8_t)m;
+  }
+  __syncthreads();
+  const int per = (C + NT - 1) / NT;
+  const int c0 = min(C, (int)threadIdx.x * per), c1 = min(C, c0 + per);
   int sz = 0;
   for (int c = c0; c < c1; ++c) sz += mask[c] ? off[c + 1] - off[c] : 0;
   int total;
@@ -473,6 +499,7 @@ __global__ void __launch_bounds__(NT) cluster_select_kernel(const ClusterParams 
     if (mask[c]) ub += off[c + 1] - off[c];
   }
   __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t* ui = p.uidx + (size_t)bg * p.nb;
   uint8_t* um = p.umask + (size_t)bg * p.nb;
   const int32_t* tk = cp.tok + (size_t)bg * cp.n_ctx;

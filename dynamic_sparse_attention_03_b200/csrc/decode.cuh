@@ -48,6 +48,7 @@ struct DecodeParams {
   float* part_ml;              // ws [B*Hq][nchmax][2]
   float* part_acc;             // ws [B*Hq][nchmax][D]
   float* scores;               // ws [B*Hq][nb] q·c
+  uint32_t* kbits;             // ws [B*Hq][ceil(nb/32)] kept blocks (or clusters) per q-head
   const __nv_bfloat16* kp;     // optional [B][Hkv][n_packed][D]: K rows in cluster order
   const __nv_bfloat16* vp;     //   (list entries below n_packed are positions in these)
   int n_packed;                // 0 when the list holds cache token ids only
@@ -109,47 +110,64 @@ __global__ void __launch_bounds__(256) decode_score_kernel(const DecodeParams p)
 }
 
 // ---------------------------------------------------------------- select
-template <int D, int GRP, int NT>
-__global__ void __launch_bounds__(NT) decode_select_kernel(const DecodeParams p) {
+// Two launches, so the top-k of every q-head runs in parallel: one CTA per
+// (batch, q-head) selects that head's blocks from its stored scores (the last
+// block always kept when force_last) and writes them as a bitmap (and the
+// optional selection outputs); one CTA per (batch, KV head) then ORs the
+// group's bitmaps into the ascending union list with a head mask per block.
+template <int NT>
+__global__ void __launch_bounds__(NT) decode_topk_kernel(const DecodeParams p) {
   extern __shared__ __align__(16) uint8_t dsm[];
+  __shared__ SelectSmem sm;
+  const int bh = blockIdx.x;   // b * Hq + h
+  const int nb = p.nb, nw = (nb + 31) >> 5;
+  float* sc = reinterpret_cast<float*>(dsm);                  // [nb]
+  int32_t* tmp = reinterpret_cast<int32_t*>(sc + nb);         // [nb]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(tmp + nb);     // [nw]
+  const float* gsc = p.scores + (size_t)bh * nb;
+  for (int x = threadIdx.x; x < nb; x += NT) sc[x] = gsc[x];
+  for (int x = threadIdx.x; x < nw; x += NT) bits[x] = 0u;
+  __syncthreads();
+  const int ncand = p.force_last ? nb - 1 : nb;
+  const int cnt = topk_ascending<NT>(sc, ncand, p.keep, 0, nb, tmp, nb, sm);
+  __syncthreads();
+  for (int x = threadIdx.x; x < cnt; x += NT) atomicOr(&bits[tmp[x] >> 5], 1u << (tmp[x] & 31));
+  if (p.sel_idx) {
+    int32_t* out = p.sel_idx + (size_t)bh * p.kcap;
+    for (int x = threadIdx.x; x < p.kcap; x += NT) out[x] = x < cnt ? tmp[x] : -1;
+  }
+  if (p.sel_cnt && threadIdx.x == 0) p.sel_cnt[bh] = cnt;
+  __syncthreads();
+  uint32_t* gb = p.kbits + (size_t)bh * nw;
+  for (int x = threadIdx.x; x < nw; x += NT) gb[x] = bits[x];
+}
+
+template <int GRP, int NT>
+__global__ void __launch_bounds__(NT) decode_union_kernel(const DecodeParams p) {
   __shared__ SelectSmem sm;
   const int bg = blockIdx.x;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
-  const int nb = p.nb;
-  constexpr int grp = GRP;
-  float* sc = reinterpret_cast<float*>(dsm);                              // [grp][nb]
-  int32_t* tmp = reinterpret_cast<int32_t*>(sc + (size_t)grp * nb);   // [nb]
-  uint8_t* mask = reinterpret_cast<uint8_t*>(tmp + nb);      // [nb]
-  const float* gsc = p.scores + ((size_t)b * p.Hq + g * grp) * nb;   // the group's rows are contiguous
-  for (int x = threadIdx.x; x < grp * nb; x += NT) sc[x] = gsc[x];
-  for (int x = threadIdx.x; x < nb; x += NT) mask[x] = 0;
-  __syncthreads();
-  const int ncand = p.force_last ? nb - 1 : nb;
-  for (int hh = 0; hh < grp; ++hh) {
-    const int cnt = topk_ascending<NT>(sc + (size_t)hh * nb, ncand, p.keep, 0, nb, tmp, nb, sm);
-    __syncthreads();
-    const int h = g * grp + hh;
-    for (int x = threadIdx.x; x < cnt; x += NT) mask[tmp[x]] |= (uint8_t)(1u << hh);
-    if (p.sel_idx) {
-      int32_t* out = p.sel_idx + ((size_t)b * p.Hq + h) * p.kcap;
-      for (int x = threadIdx.x; x < p.kcap; x += NT) out[x] = x < cnt ? tmp[x] : -1;
-    }
-    if (p.sel_cnt && threadIdx.x == 0) p.sel_cnt[(size_t)b * p.Hq + h] = cnt;
-    __syncthreads();
-  }
-  // union of the group's kept blocks, ascending, with head masks
+  const int nb = p.nb, nw = (nb + 31) >> 5;
+  const uint32_t* gb = p.kbits + ((size_t)b * p.Hq + g * GRP) * nw;   // the group's rows are contiguous
+  auto mask_of = [&](int x) {
+    uint32_t m = 0u;
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) m |= ((gb[(size_t)hh * nw + (x >> 5)] >> (x & 31)) & 1u) << hh;
+    return m;
+  };
   const int per = (nb + NT - 1) / NT;
   const int p0 = min(nb, (int)threadIdx.x * per), p1 = min(nb, p0 + per);
   int kept = 0;
-  for (int x = p0; x < p1; ++x) kept += mask[x] != 0;
+  for (int x = p0; x < p1; ++x) kept += mask_of(x) != 0u;
   int total;
   int off = block_excl_scan<NT>(kept, sm, total);
   int32_t* ui = p.uidx + (size_t)bg * nb;
   uint8_t* um = p.umask + (size_t)bg * nb;
   for (int x = p0; x < p1; ++x) {
-    if (mask[x]) {
+    const uint32_t m = mask_of(x);
+    if (m) {
       ui[off] = x;
-      um[off] = mask[x];
+      um[off] = (uint8_t)m;
       ++off;
     }
   }

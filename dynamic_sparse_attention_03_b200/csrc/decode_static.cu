@@ -90,12 +90,14 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 template <int D, int G>
 int launch(const DecodeParams& p, int B, int Hkv, int nchmax, size_t sel_smem, cudaStream_t st) {
   if (sel_smem > 48 * 1024 &&
-      cudaFuncSetAttribute(decode_select_kernel<D, G, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)sel_smem) != cudaSuccess)
+      cudaFuncSetAttribute(decode_topk_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem) !=
+          cudaSuccess)
     return DSA_ERR_CUDA;
   decode_score_kernel<D, G><<<dim3(B * Hkv, (p.nb + 63) / 64), 256, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  decode_select_kernel<D, G, 256><<<B * Hkv, 256, sel_smem, st>>>(p);
+  decode_topk_kernel<256><<<B * Hkv * G, 256, sel_smem, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  decode_union_kernel<G, 256><<<B * Hkv, 256, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (cudaFuncSetAttribute(decode_attn_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DecLayout<D>::kBytes) != cudaSuccess)
@@ -126,13 +128,14 @@ extern "C" int sparse_decode_attn_static(const void* q, const void* k_cache, con
   const int ncand = force_last ? nb - 1 : nb;
   const int count = (keep < ncand ? keep : ncand) + force_last;
   if (sel_idx && kcap < count) return DSA_ERR_CAPACITY;
-  const size_t sel_smem = (size_t)grp * nb * 4 + (size_t)nb * 4 + nb;
+  const size_t sel_smem = (size_t)nb * 8 + (size_t)((nb + 31) / 32) * 4;   // one q-head's scores, ids, bitmap
   if (sel_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
   const int nchmax = (nb + kDecChunk - 1) / kDecChunk;
-  // Scratch layout (same as the workspace of sparse_decode_attn): status word,
-  // union lists and masks, union counts, chunk partials, block scores.
+  // Scratch layout (the workspace of sparse_decode_attn): status word, per-head
+  // kept bitmaps, union lists and masks, union counts, chunk partials, block scores.
   size_t off = 0;
   const size_t o_status = off; off = up256(off + 256);
+  const size_t o_bits = off;   off = up256(off + (size_t)B * Hq * ((nb + 31) / 32) * 4);
   const size_t o_uidx = off;   off = up256(off + (size_t)B * Hkv * nb * 4);
   const size_t o_umask = off;  off = up256(off + (size_t)B * Hkv * nb);
   const size_t o_ucnt = off;   off = up256(off + (size_t)B * Hkv * 4);
@@ -147,6 +150,7 @@ extern "C" int sparse_decode_attn_static(const void* q, const void* k_cache, con
   if (cudaMemsetAsync(base + o_status, 0, 256, st) != cudaSuccess) return DSA_ERR_CUDA;
   DecodeParams p{};
   p.status = reinterpret_cast<uint32_t*>(base + o_status);
+  p.kbits = reinterpret_cast<uint32_t*>(base + o_bits);
   p.uidx = reinterpret_cast<int32_t*>(base + o_uidx);
   p.umask = base + o_umask;
   p.ucnt = reinterpret_cast<int32_t*>(base + o_ucnt);

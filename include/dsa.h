@@ -163,6 +163,10 @@ int a_shape_index(int Hq, int n, int n_sink, int n_local, int32_t* block_idx, in
  *  o          [B][Hq][d] bf16 out.
  *  sel_idx    optional [B][Hq][kcap] int32 out (ascending kept blocks),
  *             sel_cnt optional [B][Hq]; kcap >= keep + force_last when given.
+ *  Sizes: d in {64, 128}; Hq / Hkv in {1, 2, 4, 8}; S % 64 == 0 and S <= 1,600,000
+ *  or so (one q-head's block scores, ids and bitmap, 8.125 B per 64-token
+ *  block, stay under 200 KB of shared memory); larger S returns
+ *  DSA_ERR_UNSUPPORTED.
  */
 int sparse_decode_attn(const void* q, const void* k_cache, const void* v_cache, const float* centroids,
                        int B, int Hq, int Hkv, int S, int d, int keep, int force_last, float scale, void* o,
@@ -182,10 +186,11 @@ int sparse_decode_attn(const void* q, const void* k_cache, const void* v_cache, 
  *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *    Every GPU that loads the library holds the 32 MiB array until exit.
  *  - Sizes whose scratch exceeds 32 MiB are rejected with DSA_ERR_CAPACITY
- *    before any launch.  The scratch is 256 B + B·Hkv·nb·5 B (union lists and
- *    masks) + B·Hkv·4 B + B·Hq·nc·(d+2)·4 B (chunk partials, nc = ceil(nb/64))
- *    + B·Hq·nb·4 B (block scores), nb = S/64, each part rounded up to 256 B:
- *    B=16, Hq=32, Hkv=8, S=131072, d=128 needs 14.0 MB.
+ *    before any launch.  The scratch is 256 B + B·Hq·ceil(nb/32)·4 B (kept
+ *    bitmaps) + B·Hkv·nb·5 B (union lists and masks) + B·Hkv·4 B +
+ *    B·Hq·nc·(d+2)·4 B (chunk partials, nc = ceil(nb/64)) + B·Hq·nb·4 B (block
+ *    scores), nb = S/64, each part rounded up to 256 B: B=16, Hq=32, Hkv=8,
+ *    S=131072, d=128 needs 14.2 MB.
  *  - The first call on a device looks up the array's device address on that
  *    device (make the device current first); make that first call before any
  *    stream capture.  The address is kept per device context: after a device
