@@ -701,9 +701,10 @@ struct ClStreamLayout {
   static constexpr int kStage = 2 * kBlkBytes;
   static constexpr int kRed = kDecStages * kStage;              // warp partials [warp][head][D + 2]
   static constexpr int kRedBytes = kClWarps * kMaxGrp * (D + 2) * 4;
-  static constexpr int kMask = kRed + kRedBytes;                // 64 head-mask bytes per stage
-  static constexpr int kBar = kMask + kDecStages * 64;
-  static constexpr int kBytes = kBar + 2 * kDecStages * 8 + 16;
+  static constexpr int kList = kRed + kRedBytes;                // the chunk's list entries (kClChunk ints)
+  static constexpr int kMask = kList + kClChunk * 4;            // and their head masks (kClChunk bytes)
+  static constexpr int kBar = kMask + kClChunk;
+  static constexpr int kBytes = kBar + (2 * kDecStages + 1) * 8 + 16;
 };
 
 template <int D, int GRP>
@@ -723,30 +724,42 @@ __global__ void __launch_bounds__((kClWarps + 1) * 32, 1) cluster_stream_attn_ke
   const uint32_t bar0 = sb + Lay::kBar;
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (kDecStages + s); };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + Lay::kBar + 2 * kDecStages * 8);
+  const uint32_t lbar = bar0 + 8u * (2 * kDecStages);   // the chunk's list and masks landed
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsm + Lay::kBar + (2 * kDecStages + 1) * 8);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(full(s), 1);
       mbar_init(empty(s), NW);
     }
+    mbar_init(lbar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
   const AbortState ab{abort_flag, p.status};
-  const int32_t* ui = p.uidx + (size_t)bg * p.nb;
-  const uint8_t* um = p.umask + (size_t)bg * p.nb;
+  const int32_t* ui_s = reinterpret_cast<const int32_t*>(dsm + Lay::kList);   // entries e0 .. e1 - 1
+  const uint8_t* um_s = dsm + Lay::kMask;
   constexpr uint32_t kRowBytes = D * 2;
 
   if (warp == NW) {
-    // producer warp: runs of consecutive positions of each unit
+    // producer warp: the chunk's list entries and head masks come in once
+    // (two bulk copies; the list rows are padded to 16 entries, so the rounded
+    // sizes stay inside them), then the runs of consecutive positions of each
+    // unit are found in shared memory
+    if (lane == 0) {
+      const uint32_t nl = (uint32_t)((e1 - e0 + 3) & ~3) * 4u, nm = (uint32_t)((e1 - e0 + 15) & ~15);
+      mbar_arrive_expect_tx(lbar, nl + nm);
+      bulk_load(sb + Lay::kList, p.uidx + (size_t)bg * p.nb + e0, nl, lbar);
+      bulk_load(sb + Lay::kMask, p.umask + (size_t)bg * p.nb + e0, nm, lbar);
+    }
+    bool lok = mbar_wait_warp(lbar, 0, ab);
     int u = 0;
-    for (; u < nu; ++u) {
+    for (; u < nu && lok; ++u) {
       const int s = u % kDecStages;
       if (u >= kDecStages && !mbar_wait_warp(empty(s), ((u / kDecStages) - 1) & 1, ab)) break;
       const int rb = e0 + 64 * u, rows = min(64, e1 - rb);
-      const int pa = lane < rows ? ui[rb + lane] : -1;
-      const int pb = lane + 32 < rows ? ui[rb + lane + 32] : -1;
+      const int pa = lane < rows ? ui_s[64 * u + lane] : -1;
+      const int pb = lane + 32 < rows ? ui_s[64 * u + lane + 32] : -1;
       const int up_a = __shfl_up_sync(0xFFFFFFFFu, pa, 1), last_a = __shfl_sync(0xFFFFFFFFu, pa, 31);
       const int up_b = __shfl_up_sync(0xFFFFFFFFu, pb, 1);
       const int prev_b = lane == 0 ? last_a : up_b;
@@ -755,12 +768,7 @@ __global__ void __launch_bounds__((kClWarps + 1) * 32, 1) cluster_stream_attn_ke
       const bool st_a = lane < rows && (lane == 0 || pa != up_a + 1 || pa == p.n_packed);
       const bool st_b = lane + 32 < rows && (pb != prev_b + 1 || pb == p.n_packed);
       uint64_t starts = (uint64_t)__ballot_sync(0xFFFFFFFFu, st_a) | ((uint64_t)__ballot_sync(0xFFFFFFFFu, st_b) << 32);
-      // the unit's head masks ride with its rows (64 bytes, 16-byte aligned)
-      const uint32_t mbytes = (uint32_t)((rows + 15) & ~15);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(full(s), (uint32_t)rows * 2u * kRowBytes + mbytes);
-        bulk_load(sb + Lay::kMask + s * 64, um + rb, mbytes, full(s));
-      }
+      if (lane == 0) mbar_arrive_expect_tx(full(s), (uint32_t)rows * 2u * kRowBytes);
       while (starts) {   // warp-uniform
         const int r = __ffsll((long long)starts) - 1;
         starts &= starts - 1ull;
@@ -777,9 +785,11 @@ __global__ void __launch_bounds__((kClWarps + 1) * 32, 1) cluster_stream_attn_ke
       }
       __syncwarp();
     }
-    if (lane == 0)
+    if (lane == 0) {
+      if (!lok) mbar_wait_cleanup(lbar, 0, 200000000ull);
       for (int w = max(0, u - kDecStages); w < u; ++w)
         mbar_wait_cleanup(full(w % kDecStages), (w / kDecStages) & 1, 200000000ull);
+    }
     return;
   }
   // consumers: warp w takes rows 2 TPL w .. of every unit; the two half
@@ -800,15 +810,15 @@ __global__ void __launch_bounds__((kClWarps + 1) * 32, 1) cluster_stream_attn_ke
 #pragma unroll
     for (int a = 0; a < DPL; ++a) acc[hh][a] = 0.f;
   }
-  bool ok = true;
-  for (int u = 0; u < nu; ++u) {
+  bool ok = mbar_wait_warp(lbar, 0, ab);
+  for (int u = 0; u < nu && ok; ++u) {
     const int s = u % kDecStages;
     const int rb = e0 + 64 * u, rows = min(64, e1 - rb);
     if (!mbar_wait_warp(full(s), (u / kDecStages) & 1, ab)) {
       ok = false;
       break;
     }
-    const uint8_t* ms = dsm + Lay::kMask + s * 64;
+    const uint8_t* ms = um_s + 64 * u;
     uint32_t msk[TPL];
     uint32_t mor = 0u;
 #pragma unroll

@@ -220,20 +220,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(const Decod
   const size_t head_base = (size_t)bg * p.S * D;
 
   if (warp == NW) {
-    // producer: one thread streams whole K and V blocks
-    if (lane == 0) {
-      int u = 0;
-      for (; u < nu; ++u) {
-        const int s = u % kDecStages;
-        if (u >= kDecStages && !mbar_wait(empty(s), ((u / kDecStages) - 1) & 1, ab)) break;
-        const size_t off = head_base + (size_t)ui[u] * 64 * D;
+    // producer: the chunk's (at most 64) block ids come in once, two per
+    // lane, so no unit waits on a list load; lane 0 streams whole K and V
+    // blocks
+    static_assert(kDecChunk <= 64, "two list entries per producer lane");
+    const int ida = lane < nu ? ui[lane] : 0, idb = lane + 32 < nu ? ui[lane + 32] : 0;
+    int u = 0;
+    for (; u < nu; ++u) {
+      const int s = u % kDecStages;
+      if (u >= kDecStages && !mbar_wait_warp(empty(s), ((u / kDecStages) - 1) & 1, ab)) break;
+      const int blk = __shfl_sync(0xFFFFFFFFu, u < 32 ? ida : idb, u & 31);
+      if (lane == 0) {
+        const size_t off = head_base + (size_t)blk * 64 * D;
         mbar_arrive_expect_tx(full(s), 2u * Lay::kBlkBytes);
         bulk_load(sb + s * Lay::kStage, p.kc + off, Lay::kBlkBytes, full(s));
         bulk_load(sb + s * Lay::kStage + Lay::kBlkBytes, p.vc + off, Lay::kBlkBytes, full(s));
       }
+      __syncwarp();
+    }
+    if (lane == 0)
       for (int w = max(0, u - kDecStages); w < u; ++w)
         mbar_wait_cleanup(full(w % kDecStages), (w / kDecStages) & 1, 200000000ull);
-    }
     return;
   }
   // consumers: warp w takes keys 2 TPL w .. of every block; the two half
