@@ -794,21 +794,25 @@ __global__ void __launch_bounds__((kClWarps + 1) * 32, 1) cluster_stream_attn_ke
   }
   // consumers: warp w takes rows 2 TPL w .. of every unit; the two half
   // warps take alternate rows, lane%16 owns dims [DPL*(lane%16), +DPL)
-  constexpr int DPL = D / 16;
+  // (dot products and P.V updates as packed f32x2 multiply-adds on pairs of dims)
+  constexpr int DPL = D / 16, DP2 = DPL / 2;
   const int half = lane >> 4, dl = lane & 15;
-  float qv[GRP][DPL];
+  float2 qv[GRP][DP2];
 #pragma unroll
   for (int hh = 0; hh < GRP; ++hh)
 #pragma unroll
-    for (int a = 0; a < DPL; ++a)
-      qv[hh][a] = __bfloat162float(p.q[((size_t)b * p.Hq + g * GRP + hh) * D + dl * DPL + a]) * p.scale_log2;
-  float m[GRP], l[GRP], acc[GRP][DPL];
+    for (int j = 0; j < DP2; ++j) {
+      const __nv_bfloat16* qr = p.q + ((size_t)b * p.Hq + g * GRP + hh) * D + dl * DPL + 2 * j;
+      qv[hh][j] = make_float2(__bfloat162float(qr[0]) * p.scale_log2, __bfloat162float(qr[1]) * p.scale_log2);
+    }
+  float m[GRP], l[GRP];
+  float2 acc[GRP][DP2];
 #pragma unroll
   for (int hh = 0; hh < GRP; ++hh) {
     m[hh] = -INFINITY;
     l[hh] = 0.f;
 #pragma unroll
-    for (int a = 0; a < DPL; ++a) acc[hh][a] = 0.f;
+    for (int j = 0; j < DP2; ++j) acc[hh][j] = make_float2(0.f, 0.f);
   }
   bool ok = mbar_wait_warp(lbar, 0, ab);
   for (int u = 0; u < nu && ok; ++u) {
@@ -830,43 +834,36 @@ __global__ void __launch_bounds__((kClWarps + 1) * 32, 1) cluster_stream_attn_ke
     mor = __reduce_or_sync(0xFFFFFFFFu, mor);
     const uint8_t* kb = dsm + s * Lay::kStage;
     const uint8_t* vb = kb + Lay::kBlkBytes;
-    float kf[TPL][DPL], vf[TPL][DPL];
+    float2 kf[TPL][DP2], vf[TPL][DP2];
 #pragma unroll
     for (int it = 0; it < TPL; ++it) {
       const int key = 2 * TPL * warp + 2 * it + half;
-      const bool valid = key < rows;   // rows past the unit's end hold stale bytes: never used
+      // rows past the unit's end hold stale bytes (the stage has room for 64
+      // rows, so the loads stay inside it): their words are zeroed
+      const uint32_t keep = key < rows ? 0xFFFFFFFFu : 0u;
+      if constexpr (DPL == 8) {
+        uint4 kr = *reinterpret_cast<const uint4*>(kb + key * kRowBytes + dl * 16);
+        uint4 vr = *reinterpret_cast<const uint4*>(vb + key * kRowBytes + dl * 16);
+        kr.x &= keep; kr.y &= keep; kr.z &= keep; kr.w &= keep;
+        vr.x &= keep; vr.y &= keep; vr.z &= keep; vr.w &= keep;
+        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
 #pragma unroll
-      for (int a = 0; a < DPL; ++a) {
-        kf[it][a] = 0.f;
-        vf[it][a] = 0.f;
-      }
-      if (valid) {
-        if constexpr (DPL == 8) {
-          const uint4 kr = *reinterpret_cast<const uint4*>(kb + key * kRowBytes + dl * 16);
-          const uint4 vr = *reinterpret_cast<const uint4*>(vb + key * kRowBytes + dl * 16);
-          const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
-          const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
+        for (int j = 0; j < 4; ++j) {
+          kf[it][j] = __bfloat1622float2(k2[j]);
+          vf[it][j] = __bfloat1622float2(v2[j]);
+        }
+      } else {
+        uint2 kr = *reinterpret_cast<const uint2*>(kb + key * kRowBytes + dl * 8);
+        uint2 vr = *reinterpret_cast<const uint2*>(vb + key * kRowBytes + dl * 8);
+        kr.x &= keep; kr.y &= keep;
+        vr.x &= keep; vr.y &= keep;
+        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
 #pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            const float2 kk = __bfloat1622float2(k2[a]), vv = __bfloat1622float2(v2[a]);
-            kf[it][2 * a] = kk.x;
-            kf[it][2 * a + 1] = kk.y;
-            vf[it][2 * a] = vv.x;
-            vf[it][2 * a + 1] = vv.y;
-          }
-        } else {
-          const uint2 kr = *reinterpret_cast<const uint2*>(kb + key * kRowBytes + dl * 8);
-          const uint2 vr = *reinterpret_cast<const uint2*>(vb + key * kRowBytes + dl * 8);
-          const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
-          const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
-#pragma unroll
-          for (int a = 0; a < 2; ++a) {
-            const float2 kk = __bfloat1622float2(k2[a]), vv = __bfloat1622float2(v2[a]);
-            kf[it][(2 * a) % DPL] = kk.x;
-            kf[it][(2 * a + 1) % DPL] = kk.y;
-            vf[it][(2 * a) % DPL] = vv.x;
-            vf[it][(2 * a + 1) % DPL] = vv.y;
-          }
+        for (int j = 0; j < 2; ++j) {
+          kf[it][j % DP2] = __bfloat1622float2(k2[j]);
+          vf[it][j % DP2] = __bfloat1622float2(v2[j]);
         }
       }
     }
@@ -879,9 +876,10 @@ __global__ void __launch_bounds__((kClWarps + 1) * 32, 1) cluster_stream_attn_ke
       float sc[TPL];
 #pragma unroll
       for (int it = 0; it < TPL; ++it) {
-        float d0 = 0.f;
+        float2 t = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int a = 0; a < DPL; ++a) d0 = fmaf(qv[hh][a], kf[it][a], d0);
+        for (int j = 0; j < DP2; ++j) t = ffma2(qv[hh][j], kf[it][j], t);
+        float d0 = t.x + t.y;
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) d0 += __shfl_xor_sync(0xFFFFFFFFu, d0, o);
         sc[it] = ((msk[it] >> hh) & 1u) ? d0 : -INFINITY;
@@ -895,13 +893,13 @@ __global__ void __launch_bounds__((kClWarps + 1) * 32, 1) cluster_stream_attn_ke
       const float alpha = ex2_approx(m[hh] - mn);   // m = -inf -> 0
       float ls = 0.f;
 #pragma unroll
-      for (int a = 0; a < DPL; ++a) acc[hh][a] *= alpha;
+      for (int j = 0; j < DP2; ++j) acc[hh][j] = fmul2(acc[hh][j], make_float2(alpha, alpha));
 #pragma unroll
       for (int it = 0; it < TPL; ++it) {
         const float pe = ex2_approx(sc[it] - mn);   // -inf -> 0
         ls += pe;
 #pragma unroll
-        for (int a = 0; a < DPL; ++a) acc[hh][a] = fmaf(pe, vf[it][a], acc[hh][a]);
+        for (int j = 0; j < DP2; ++j) acc[hh][j] = ffma2(make_float2(pe, pe), vf[it][j], acc[hh][j]);
       }
       l[hh] = l[hh] * alpha + ls;
       m[hh] = mn;
@@ -913,11 +911,17 @@ __global__ void __launch_bounds__((kClWarps + 1) * 32, 1) cluster_stream_attn_ke
   for (int hh = 0; hh < GRP; ++hh) {
     l[hh] += __shfl_xor_sync(0xFFFFFFFFu, l[hh], 16);
 #pragma unroll
-    for (int a = 0; a < DPL; ++a) acc[hh][a] += __shfl_xor_sync(0xFFFFFFFFu, acc[hh][a], 16);
+    for (int j = 0; j < DP2; ++j) {
+      acc[hh][j].x += __shfl_xor_sync(0xFFFFFFFFu, acc[hh][j].x, 16);
+      acc[hh][j].y += __shfl_xor_sync(0xFFFFFFFFu, acc[hh][j].y, 16);
+    }
     float* r = red + ((size_t)warp * kMaxGrp + hh) * (D + 2);
     if (half == 0) {
 #pragma unroll
-      for (int a = 0; a < DPL; ++a) r[dl * DPL + a] = acc[hh][a];
+      for (int j = 0; j < DP2; ++j) {
+        r[dl * DPL + 2 * j] = acc[hh][j].x;
+        r[dl * DPL + 2 * j + 1] = acc[hh][j].y;
+      }
     }
     if (lane == 0) {
       r[D] = m[hh];

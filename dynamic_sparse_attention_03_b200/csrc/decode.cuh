@@ -245,21 +245,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(const Decod
   }
   // consumers: warp w takes keys 2 TPL w .. of every block; the two half
   // warps take alternate keys, lane%16 owns dims [DPL*(lane%16), +DPL).
-  constexpr int DPL = D / 16;            // dims per lane (8 at d=128, 4 at d=64)
+  // (dot products and P.V updates as packed f32x2 multiply-adds on pairs of dims)
+  constexpr int DPL = D / 16, DP2 = DPL / 2;   // dims per lane (8 at d=128, 4 at d=64)
   const int half = lane >> 4, dl = lane & 15;
-  float qv[GRP][DPL];
+  float2 qv[GRP][DP2];
 #pragma unroll
   for (int hh = 0; hh < grp; ++hh)
 #pragma unroll
-    for (int a = 0; a < DPL; ++a)
-      qv[hh][a] = __bfloat162float(p.q[((size_t)b * p.Hq + g * grp + hh) * D + dl * DPL + a]) * p.scale_log2;
-  float m[GRP], l[GRP], acc[GRP][DPL];
+    for (int j = 0; j < DP2; ++j) {
+      const __nv_bfloat16* qr = p.q + ((size_t)b * p.Hq + g * grp + hh) * D + dl * DPL + 2 * j;
+      qv[hh][j] = make_float2(__bfloat162float(qr[0]) * p.scale_log2, __bfloat162float(qr[1]) * p.scale_log2);
+    }
+  float m[GRP], l[GRP];
+  float2 acc[GRP][DP2];
 #pragma unroll
   for (int hh = 0; hh < GRP; ++hh) {
     m[hh] = -INFINITY;
     l[hh] = 0.f;
 #pragma unroll
-    for (int a = 0; a < DPL; ++a) acc[hh][a] = 0.f;
+    for (int j = 0; j < DP2; ++j) acc[hh][j] = make_float2(0.f, 0.f);
   }
   bool ok = true;
   for (int u = 0; u < nu; ++u) {
@@ -269,21 +273,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(const Decod
     const uint8_t* kb = dsm + s * Lay::kStage;
     const uint8_t* vb = kb + Lay::kBlkBytes;
     // TPL keys per lane: key = 2 TPL warp + 2 it + half
-    float kf[TPL][DPL], vf[TPL][DPL];
+    float2 kf[TPL][DP2], vf[TPL][DP2];
 #pragma unroll
     for (int it = 0; it < TPL; ++it) {
       const int key = 2 * TPL * warp + 2 * it + half;
-      if (DPL == 8) {
+      if constexpr (DPL == 8) {
         const uint4 kr = *reinterpret_cast<const uint4*>(kb + key * D * 2 + dl * 16);
         const uint4 vr = *reinterpret_cast<const uint4*>(vb + key * D * 2 + dl * 16);
         const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
         const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          const float2 kk = __bfloat1622float2(k2[a]);
-          const float2 vv = __bfloat1622float2(v2[a]);
-          kf[it][(2 * a) % DPL] = kk.x; kf[it][(2 * a + 1) % DPL] = kk.y;
-          vf[it][(2 * a) % DPL] = vv.x; vf[it][(2 * a + 1) % DPL] = vv.y;
+        for (int j = 0; j < 4; ++j) {
+          kf[it][j] = __bfloat1622float2(k2[j]);
+          vf[it][j] = __bfloat1622float2(v2[j]);
         }
       } else {
         const uint2 kr = *reinterpret_cast<const uint2*>(kb + key * D * 2 + dl * 8);
@@ -291,11 +293,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(const Decod
         const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
         const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
-          const float2 kk = __bfloat1622float2(k2[a]);
-          const float2 vv = __bfloat1622float2(v2[a]);
-          kf[it][(2 * a) % DPL] = kk.x; kf[it][(2 * a + 1) % DPL] = kk.y;
-          vf[it][(2 * a) % DPL] = vv.x; vf[it][(2 * a + 1) % DPL] = vv.y;
+        for (int j = 0; j < 2; ++j) {
+          kf[it][j % DP2] = __bfloat1622float2(k2[j]);
+          vf[it][j % DP2] = __bfloat1622float2(v2[j]);
         }
       }
     }
@@ -308,9 +308,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(const Decod
       float sc[TPL];
 #pragma unroll
       for (int it = 0; it < TPL; ++it) {
-        float d0 = 0.f;
+        float2 t = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int a = 0; a < DPL; ++a) d0 = fmaf(qv[hh][a], kf[it][a], d0);
+        for (int j = 0; j < DP2; ++j) t = ffma2(qv[hh][j], kf[it][j], t);
+        float d0 = t.x + t.y;
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) d0 += __shfl_xor_sync(0xFFFFFFFFu, d0, o);
         sc[it] = d0;
@@ -323,13 +324,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(const Decod
       const float alpha = ex2_approx(m[hh] - mn);   // m = -inf -> 0
       float ls = 0.f;
 #pragma unroll
-      for (int a = 0; a < DPL; ++a) acc[hh][a] *= alpha;
+      for (int j = 0; j < DP2; ++j) acc[hh][j] = fmul2(acc[hh][j], make_float2(alpha, alpha));
 #pragma unroll
       for (int it = 0; it < TPL; ++it) {
         const float pe = ex2_approx(sc[it] - mn);
         ls += pe;
 #pragma unroll
-        for (int a = 0; a < DPL; ++a) acc[hh][a] = fmaf(pe, vf[it][a], acc[hh][a]);
+        for (int j = 0; j < DP2; ++j) acc[hh][j] = ffma2(make_float2(pe, pe), vf[it][j], acc[hh][j]);
       }
       l[hh] = l[hh] * alpha + ls;
       m[hh] = mn;
@@ -341,11 +342,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_attn_kernel(const Decod
   for (int hh = 0; hh < grp; ++hh) {
     l[hh] += __shfl_xor_sync(0xFFFFFFFFu, l[hh], 16);
 #pragma unroll
-    for (int a = 0; a < DPL; ++a) acc[hh][a] += __shfl_xor_sync(0xFFFFFFFFu, acc[hh][a], 16);
+    for (int j = 0; j < DP2; ++j) {
+      acc[hh][j].x += __shfl_xor_sync(0xFFFFFFFFu, acc[hh][j].x, 16);
+      acc[hh][j].y += __shfl_xor_sync(0xFFFFFFFFu, acc[hh][j].y, 16);
+    }
     float* r = red + ((size_t)warp * kMaxGrp + hh) * (D + 2);
     if (half == 0) {
 #pragma unroll
-      for (int a = 0; a < DPL; ++a) r[dl * DPL + a] = acc[hh][a];
+      for (int j = 0; j < DP2; ++j) {
+        r[dl * DPL + 2 * j] = acc[hh][j].x;
+        r[dl * DPL + 2 * j + 1] = acc[hh][j].y;
+      }
     }
     if (lane == 0) {
       r[D] = m[hh];
