@@ -406,6 +406,13 @@ int vertical_slash_index(const void* q, const void* k, int Hq, int Hkv, int n, i
   p.slash = static_cast<float*>(c.take((size_t)Hq * n * 4));
   p.vsel = vert_idx ? vert_idx : static_cast<int32_t*>(c.take((size_t)Hq * n_vert * 4));
   p.ssel = slash_off ? slash_off : static_cast<int32_t*>(c.take((size_t)Hq * n_slash * 4));
+  // slice survivors: at most min(e, slice length) per slice and kind
+  const int ecap = std::max(1, std::min(std::max(n_vert - 64, n_slash - 1), (n + kVSParts - 1) / kVSParts));
+  p.cand_id = static_cast<int32_t*>(c.take((size_t)Hq * 2 * kVSParts * ecap * 4));
+  p.cand_cnt = static_cast<int32_t*>(c.take((size_t)Hq * 2 * kVSParts * 4));
+  p.cand_val = static_cast<float*>(c.take((size_t)Hq * 2 * kVSParts * ecap * 4));
+  p.cand_gid = static_cast<int32_t*>(c.take((size_t)Hq * 2 * kVSParts * ecap * 4));
+  p.ecap = ecap;
   p.dbits = static_cast<uint32_t*>(c.take((size_t)Hq * ((nQB + 31) / 32) * 4));
   p.dlist = static_cast<int32_t*>(c.take((size_t)Hq * nQB * 4));
   p.dcount = static_cast<int32_t*>(c.take((size_t)Hq * 4));
@@ -450,12 +457,14 @@ int vertical_slash_index(const void* q, const void* k, int Hq, int Hkv, int n, i
     vs_score_kernel<64, 1><<<gl, 256, VSScoreLayout<64>::kSmemAlloc, st>>>(tq, tk, p);
   }
   if ((rc = launch_check())) return rc;
-  vs_lse_kernel<<<Hq, 64, 0, st>>>(p);
+  vs_lse_kernel<<<Hq * 64, 128, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
   if (d == 128) vs_score_kernel<128, 2><<<gl, 256, VSScoreLayout<128>::kSmemAlloc, st>>>(tq, tk, p);
   else vs_score_kernel<64, 2><<<gl, 256, VSScoreLayout<64>::kSmemAlloc, st>>>(tq, tk, p);
   if ((rc = launch_check())) return rc;
   vs_slash_kernel<<<dim3((n + 255) / 256, Hq), 256, 0, st>>>(p);
+  if ((rc = launch_check())) return rc;
+  vs_topk_part_kernel<256><<<dim3(Hq, 2, kVSParts), 256, 0, st>>>(p);
   if ((rc = launch_check())) return rc;
   vs_topk_kernel<1024><<<dim3(Hq, 2), 1024, 0, st>>>(p);
   if ((rc = launch_check())) return rc;

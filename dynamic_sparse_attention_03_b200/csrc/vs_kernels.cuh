@@ -27,6 +27,7 @@ namespace dsa {
 
 constexpr int kVSTile = 128;              // keys per CTA of the two score passes
 constexpr int kVSDiag = kVSTile + 63;     // diagonal offsets one tile touches (191)
+constexpr int kVSParts = 8;               // slices of a head's scores ranked apart before the final top-k
 
 struct VSParams {
   const __nv_bfloat16* q;
@@ -39,6 +40,11 @@ struct VSParams {
   float* slash;       // [Hq][n]
   int32_t* vsel;      // [Hq][n_vert]
   int32_t* ssel;      // [Hq][n_slash]
+  int32_t* cand_id;   // [Hq][2][kVSParts][ecap] slice top-k: candidate indices, ascending
+  int32_t* cand_cnt;  // [Hq][2][kVSParts]
+  float* cand_val;    // [Hq][2][kVSParts * ecap] the candidates gathered in index order
+  int32_t* cand_gid;  // [Hq][2][kVSParts * ecap]
+  int ecap;
   uint32_t* dbits;    // [Hq][ceil(nQB/32)] block distances reached by kept offsets
   int32_t* dlist;     // [Hq][nQB] the same distances, ascending
   int32_t* dcount;    // [Hq]
@@ -233,18 +239,46 @@ __global__ void __launch_bounds__(256, 2)
   }
 }
 
-// Per (head, row): combine the tile partials in tile order -> lse (log2 domain).
-__global__ void __launch_bounds__(64) vs_lse_kernel(const VSParams p) {
-  const int h = blockIdx.x, r = threadIdx.x;
-  const float* pp = p.part + ((size_t)h * p.ntiles * 64 + r) * 2;
-  float M = -INFINITY;
-  for (int t = 0; t < p.ntiles; ++t) M = fmaxf(M, pp[(size_t)t * 128]);
-  float L = 0.f;
-  for (int t = 0; t < p.ntiles; ++t) {
-    const float mt = pp[(size_t)t * 128];
-    if (mt != -INFINITY) L += pp[(size_t)t * 128 + 1] * exp2f(mt - M);
+// Per (head, row): combine the tile partials -> lse (log2 domain).  One CTA
+// per (head, row): each thread folds the tiles t = tid, tid + 128, ... in that
+// order, then the threads' (max, sum) pairs are merged by a fixed tree
+// (lanes by xor-shuffles, whose two sides compute the same sum, then the four
+// warps in order), so the result does not depend on timing.
+__device__ __forceinline__ void lse_merge(float& M, float& L, float M2, float L2) {
+  if (M2 == -INFINITY) return;
+  if (M == -INFINITY) {
+    M = M2;
+    L = L2;
+  } else if (M2 > M) {
+    L = L * exp2f(M - M2) + L2;
+    M = M2;
+  } else {
+    L += L2 * exp2f(M2 - M);
   }
-  p.lse2[h * 64 + r] = M + log2f(L);
+}
+
+__global__ void __launch_bounds__(128) vs_lse_kernel(const VSParams p) {
+  __shared__ float wm[4], wl[4];
+  const int h = blockIdx.x >> 6, r = blockIdx.x & 63;
+  const float* pp = p.part + ((size_t)h * p.ntiles * 64 + r) * 2;
+  float M = -INFINITY, L = 0.f;
+  for (int t = threadIdx.x; t < p.ntiles; t += 128) lse_merge(M, L, pp[(size_t)t * 128], pp[(size_t)t * 128 + 1]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float M2 = __shfl_xor_sync(0xFFFFFFFFu, M, o), L2 = __shfl_xor_sync(0xFFFFFFFFu, L, o);
+    lse_merge(M, L, M2, L2);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    wm[threadIdx.x >> 5] = M;
+    wl[threadIdx.x >> 5] = L;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    M = wm[0];
+    L = wl[0];
+    for (int w = 1; w < 4; ++w) lse_merge(M, L, wm[w], wl[w]);
+    p.lse2[h * 64 + r] = M + log2f(L);
+  }
 }
 
 // slash[o] = sum of the (at most two) tile partials covering offset o, in tile order.
@@ -264,19 +298,68 @@ __global__ void __launch_bounds__(256) vs_slash_kernel(const VSParams p) {
   p.slash[(size_t)h * p.n + o] = s;
 }
 
-// Top columns (first 64 forced) and top offsets (offset 0 forced) per head.
+// Top columns (first 64 forced) and top offsets (offset 0 forced) per head,
+// in two launches.  The candidates (columns >= 64, offsets >= 1) of a head are
+// cut into kVSParts slices and each slice keeps its own top e (the same order:
+// higher score first, equal scores to the lower index); an element of the
+// head's top e is beaten by fewer than e others, so it is in its slice's top e
+// too.  The final top e is then taken over the slices' survivors gathered in
+// index order, which the same order ranks exactly as it ranks the whole row.
+template <int NT>
+__global__ void __launch_bounds__(NT) vs_topk_part_kernel(const VSParams p) {
+  __shared__ SelectSmem sm;
+  const int h = blockIdx.x, kind = blockIdx.y, part = blockIdx.z;
+  const int nf = kind == 0 ? min(64, p.n) : 1;   // ids always kept
+  const float* src = (kind == 0 ? p.vert : p.slash) + (size_t)h * p.n + nf;
+  const int L = p.n - nf;
+  const int e = (kind == 0 ? p.n_vert : p.n_slash) - nf;
+  const int per = (L + kVSParts - 1) / kVSParts;
+  const int a = min(L, part * per), b = min(L, a + per);
+  const size_t slot = ((size_t)h * 2 + kind) * kVSParts + part;
+  int32_t* out = p.cand_id + slot * p.ecap;
+  const int cnt = topk_ascending<NT>(src + a, b - a, e, 0, b - a, out, p.ecap, sm);
+  __syncthreads();
+  for (int j = threadIdx.x; j < cnt; j += NT) out[j] += a;   // slice positions -> candidate indices
+  if (threadIdx.x == 0) p.cand_cnt[slot] = cnt;
+}
+
 template <int NT>
 __global__ void __launch_bounds__(NT) vs_topk_kernel(const VSParams p) {
   __shared__ SelectSmem sm;
-  const int h = blockIdx.x;
-  if (blockIdx.y == 0) {
-    const int nf = min(64, p.n);
-    topk_ascending<NT>(p.vert + (size_t)h * p.n + nf, p.n - nf, p.n_vert - nf, nf, p.n,
-                       p.vsel + (size_t)h * p.n_vert, p.n_vert, sm);
-  } else {
-    topk_ascending<NT>(p.slash + (size_t)h * p.n + 1, p.n - 1, p.n_slash - 1, 1, p.n,
-                       p.ssel + (size_t)h * p.n_slash, p.n_slash, sm);
+  __shared__ int base[kVSParts + 1];
+  const int h = blockIdx.x, kind = blockIdx.y;
+  const int nf = kind == 0 ? min(64, p.n) : 1;
+  const float* src = (kind == 0 ? p.vert : p.slash) + (size_t)h * p.n + nf;
+  const int e = (kind == 0 ? p.n_vert : p.n_slash) - nf;
+  const size_t hk = (size_t)h * 2 + kind;
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int y = 0; y < kVSParts; ++y) {
+      base[y] = acc;
+      acc += p.cand_cnt[hk * kVSParts + y];
+    }
+    base[kVSParts] = acc;
   }
+  __syncthreads();
+  const int Lc = base[kVSParts];
+  float* cv = p.cand_val + hk * kVSParts * p.ecap;
+  int32_t* ci = p.cand_gid + hk * kVSParts * p.ecap;
+  for (int y = 0; y < kVSParts; ++y) {
+    const int32_t* ids = p.cand_id + (hk * kVSParts + y) * p.ecap;
+    const int c = base[y + 1] - base[y];
+    for (int j = threadIdx.x; j < c; j += NT) {
+      const int id = ids[j];
+      ci[base[y] + j] = id;
+      cv[base[y] + j] = src[id];
+    }
+  }
+  __syncthreads();
+  int32_t* out = kind == 0 ? p.vsel + (size_t)h * p.n_vert : p.ssel + (size_t)h * p.n_slash;
+  const int cap = kind == 0 ? p.n_vert : p.n_slash;
+  for (int j = threadIdx.x; j < nf; j += NT) out[j] = j;   // the forced ids come first
+  const int cnt = topk_ascending<NT>(cv, Lc, e, 0, Lc, out + nf, cap - nf, sm);
+  __syncthreads();
+  for (int j = threadIdx.x; j < cnt && j < cap - nf; j += NT) out[nf + j] = ci[out[nf + j]] + nf;
 }
 
 // Block distances of a head's kept offsets: a kept offset o reaches key
