@@ -273,6 +273,24 @@ def test_vs_index_plan_and_attention_small(n):
     check_attention(o, refo, "vs small")
 
 
+def test_vs_index_exact_ties_take_the_lower_columns():
+    """Zero keys make every logit 0, so each of the last 64 rows spreads its
+    weight evenly over its causal keys and every column before those rows gets
+    the same sum, bit for bit (the same values added in the same order).  The
+    kept columns must then be the lowest ones (MInference 1.0 page, method
+    section: the top vertical lines; ties to the lower index), also when the
+    kept count spans several of the slices the top-k ranks apart first."""
+    n, Hq, Hkv, d = 8192, 2, 1, 128
+    w = synth.make_prefill("llama3-8b-128k-vs", device=DEV, n=n, Hq=Hq, Hkv=Hkv, d=d, seed=23)
+    k0 = torch.zeros_like(w.k)
+    for n_vert in (700, 2500):
+        res = dsa.vertical_slash_index(w.q, k0, n_vert, 64)
+        torch.cuda.synchronize()
+        vi = res["vert_idx"].cpu().numpy()
+        for h in range(Hq):
+            assert vi[h].tolist() == list(range(n_vert)), (n_vert, h)
+
+
 # ---------------------------------------------------------------- decode
 
 @pytest.mark.parametrize("B,Hq,Hkv,S,d,keep", [(2, 8, 2, 8192, 128, 32), (3, 4, 4, 4096, 64, 10), (1, 8, 1, 2048, 128, 100)])
