@@ -8,15 +8,17 @@
 //  decode_score_kernel: q·c for every (batch, q-head, block), 64 centroid
 //    blocks of one (batch, KV head) per CTA, each centroid row read once for
 //    the group's q-heads.
-//  decode_select_kernel: one CTA per (batch, KV head): top `keep` per q-head of
-//    the group (ties to the lower block) plus the last block, and the union of
-//    the group's kept blocks with a per-block head mask.
+//  decode_topk_kernel: one CTA per (batch, q-head): the head's top `keep`
+//    blocks (ties to the lower block) plus the last block, as a bitmap.
+//  decode_union_kernel: one CTA per (batch, KV head): the union of the group's
+//    bitmaps as a block list with a per-block head mask.
 //  decode_attn_kernel: one CTA per (batch, KV head, chunk of union blocks).
-//    One producer thread streams whole 64-token K and V blocks (contiguous
-//    16 KB each at d = 128) into a 4-stage shared-memory ring with bulk copies;
-//    4 consumer warps score the block for every q-head that kept it, keep an
-//    online softmax per (warp, head), and merge into one partial per chunk.
-//    Each K/V block is read from HBM once for the whole GQA group.
+//    A producer warp streams whole 64-token K and V blocks (contiguous 16 KB
+//    each at d = 128) into a 4-stage shared-memory ring with bulk copies;
+//    8 consumer warps score the block for every q-head that kept it (packed
+//    f32x2 multiply-adds), keep an online softmax per (warp, head), and merge
+//    into one partial per chunk.  Each K/V block is read from HBM once for the
+//    whole GQA group.
 //  decode_combine_kernel: merges the chunk partials of each (batch, q-head).
 #pragma once
 
