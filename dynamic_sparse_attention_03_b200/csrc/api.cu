@@ -232,8 +232,8 @@ int launch_cluster_decode(const ClusterParams& cp, int B, int Hkv, int nchmax, s
   cluster_topk_kernel<256><<<B * Hkv * G, 256, sel_smem, st>>>(cp);
   if ((rc = launch_check())) return rc;
   const size_t uni_smem = (size_t)(cp.C + 1) * 4 + (size_t)cp.C * 5;
-  if ((rc = set_smem(cluster_union_kernel<G, 256>, uni_smem))) return rc;
-  cluster_union_kernel<G, 256><<<B * Hkv, 256, uni_smem, st>>>(cp);
+  if ((rc = set_smem(cluster_union_kernel<G, 1024>, uni_smem))) return rc;
+  cluster_union_kernel<G, 1024><<<B * Hkv, 1024, uni_smem, st>>>(cp);
   if ((rc = launch_check())) return rc;
   if (cp.dp.n_packed > 0) {
     if ((rc = set_smem(cluster_stream_attn_kernel<D, G>, ClStreamLayout<D>::kBytes))) return rc;
