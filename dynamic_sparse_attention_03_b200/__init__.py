@@ -155,6 +155,10 @@ class Workspace:
 
     def ensure(self, nbytes: int) -> torch.Tensor:
         if self.buf.numel() < nbytes:
+            # the old buffer may still be in use by calls queued on any stream:
+            # let them finish before its memory can be handed out again (growth
+            # happens on the first calls of a size, not in steady state)
+            torch.cuda.synchronize(self.device)
             self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
         return self.buf
 
