@@ -60,7 +60,10 @@ def test_tiny_attention_matches_oracle():
 
 # ---------------------------------------------------------------- block-sparse, GQA
 
-@pytest.mark.parametrize("n,d,Hq,Hkv,rho", [(4096, 128, 8, 2, 0.10), (2048, 64, 4, 4, 0.25), (3072, 128, 6, 2, 0.5)])
+# GQA groups of 4, 1 and 3 q-heads per KV head, and 8 and 5 (two work items
+# per KV head and query block: four heads each, or four and one)
+@pytest.mark.parametrize("n,d,Hq,Hkv,rho", [(4096, 128, 8, 2, 0.10), (2048, 64, 4, 4, 0.25), (3072, 128, 6, 2, 0.5),
+                                            (2048, 128, 16, 2, 0.2), (2048, 64, 10, 2, 0.3)])
 def test_block_index_and_attention(n, d, Hq, Hkv, rho):
     w = synth.make_prefill("llama3-8b-32k-bs10", device=DEV, n=n, Hq=Hq, Hkv=Hkv, d=d, seed=7 + n)
     bi, bc = dsa.sparse_index_estimate(w.q, w.k, keep_ratio=rho)
@@ -233,9 +236,9 @@ def test_attention_invariants():
 
 # ---------------------------------------------------------------- vertical-slash
 
-@pytest.mark.parametrize("n", [2048, 1984])
-def test_vs_index_plan_and_attention_small(n):
-    Hq, Hkv, d = 4, 2, 128
+@pytest.mark.parametrize("n,Hq,Hkv", [(2048, 4, 2), (1984, 4, 2), (2048, 16, 2)])
+def test_vs_index_plan_and_attention_small(n, Hq, Hkv):
+    d = 128
     w = synth.make_prefill("llama3-8b-128k-vs", device=DEV, n=n, Hq=Hq, Hkv=Hkv, d=d, seed=21)
     n_vert, n_slash = 200, 300
     res = dsa.vertical_slash_index(w.q, w.k, n_vert, n_slash)
