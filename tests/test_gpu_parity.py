@@ -63,7 +63,8 @@ def test_tiny_attention_matches_oracle():
 # GQA groups of 4, 1 and 3 q-heads per KV head, and 8 and 5 (two work items
 # per KV head and query block: four heads each, or four and one)
 @pytest.mark.parametrize("n,d,Hq,Hkv,rho", [(4096, 128, 8, 2, 0.10), (2048, 64, 4, 4, 0.25), (3072, 128, 6, 2, 0.5),
-                                            (2048, 128, 16, 2, 0.2), (2048, 64, 10, 2, 0.3)])
+                                            (2048, 128, 16, 2, 0.2), (2048, 64, 10, 2, 0.3),
+                                            (9024, 128, 4, 1, 0.15)])   # 141 query blocks: ragged row tile and key chunk
 def test_block_index_and_attention(n, d, Hq, Hkv, rho):
     w = synth.make_prefill("llama3-8b-32k-bs10", device=DEV, n=n, Hq=Hq, Hkv=Hkv, d=d, seed=7 + n)
     bi, bc = dsa.sparse_index_estimate(w.q, w.k, keep_ratio=rho)
