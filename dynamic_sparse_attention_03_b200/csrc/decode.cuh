@@ -60,11 +60,43 @@ struct DecodeParams {
 };
 
 // ---------------------------------------------------------------- scores
+// Sums C per-lane values over the 32 lanes of a warp and leaves them spread
+// over the lanes: each round exchanges half of a lane's values with the lane
+// `off` away and adds (the lane keeps the half its bit `off` picks), so the
+// 5 rounds take C - 1 shuffles instead of 5 C.  Afterwards lane L holds the
+// sums of values L*(C/32) .. L*(C/32) + C/32 - 1 (C >= 32), or of value
+// L / (32/C) (C < 32; the 32/C lanes of a group hold the same sum).
+template <int C>
+__device__ __forceinline__ void warp_sum_spread(float (&v)[C], int lane) {
+  int n = C;   // values a lane still holds (a constant once the loop is unrolled)
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const bool hi = (lane & off) != 0;
+      const int h = n / 2;
+#pragma unroll
+      for (int i = 0; i < C / 2; ++i) {
+        if (i < h) {
+          const float keep = hi ? v[i + h] : v[i];
+          const float send = hi ? v[i] : v[i + h];
+          v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
+        }
+      }
+      n = h;
+    } else {
+      v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], off);
+    }
+  }
+}
+
 // One CTA of 8 warps per (batch x KV head, 64 centroid blocks): each warp
-// scores 8 blocks for the group's q-heads, loading its 8 rows together.
+// scores 8 blocks for the group's q-heads, loading its 8 rows together; the
+// 8 x GRP dot products are summed over the warp with warp_sum_spread, so
+// lane-groups of the warp store the scores of one head's 8 blocks side by side.
 template <int D, int GRP>
 __global__ void __launch_bounds__(256) decode_score_kernel(const DecodeParams p) {
   constexpr int PER = D / 32;
+  constexpr int C = 8 * GRP;                 // (block, head) dot products per warp
   const int bg = blockIdx.x, t0 = blockIdx.y * 64;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -96,17 +128,27 @@ __global__ void __launch_bounds__(256) decode_score_kernel(const DecodeParams p)
       for (int a = 0; a < PER; ++a) cv[r][a] = 0.f;
     }
   }
+  // this lane's share of every (block r, head hh) dot product, value r*GRP + hh
+  float s[C];
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int t = t0 + warp * 8 + r;
+  for (int r = 0; r < 8; ++r)
 #pragma unroll
     for (int hh = 0; hh < GRP; ++hh) {
-      float s = 0.f;
+      float acc = 0.f;
 #pragma unroll
-      for (int a = 0; a < PER; ++a) s = fmaf(qreg[hh][a], cv[r][a], s);
+      for (int a = 0; a < PER; ++a) acc = fmaf(qreg[hh][a], cv[r][a], acc);
+      s[r * GRP + hh] = acc;
+    }
+  warp_sum_spread<C>(s, lane);
+  constexpr int HOLD = C >= 32 ? C / 32 : 1;   // sums this lane holds
+  constexpr int REP = C >= 32 ? 1 : 32 / C;    // lanes holding the same sum
+  if (lane % REP == 0) {
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-      if (lane == 0 && t < p.nb) p.scores[((size_t)b * p.Hq + g * GRP + hh) * p.nb + t] = s;
+    for (int j = 0; j < HOLD; ++j) {
+      const int idx = (C >= 32) ? lane * HOLD + j : lane / REP;
+      const int r = idx / GRP, hh = idx % GRP;
+      const int t = t0 + warp * 8 + r;
+      if (t < p.nb) p.scores[((size_t)b * p.Hq + g * GRP + hh) * p.nb + t] = s[j];
     }
   }
 }
