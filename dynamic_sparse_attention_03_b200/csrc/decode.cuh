@@ -63,7 +63,7 @@ struct DecodeParams {
 // Sums C per-lane values over the 32 lanes of a warp and leaves them spread
 // over the lanes: each round exchanges half of a lane's values with the lane
 // `off` away and adds (the lane keeps the half its bit `off` picks), so the
-// 5 rounds take C - 1 shuffles instead of 5 C.  Afterwards lane L holds the
+// 5 rounds take about C shuffles instead of 5 C.  Afterwards lane L holds the
 // sums of values L*(C/32) .. L*(C/32) + C/32 - 1 (C >= 32), or of value
 // L / (32/C) (C < 32; the 32/C lanes of a group hold the same sum).
 template <int C>
@@ -91,8 +91,8 @@ __device__ __forceinline__ void warp_sum_spread(float (&v)[C], int lane) {
 
 // One CTA of 8 warps per (batch x KV head, 64 centroid blocks): each warp
 // scores 8 blocks for the group's q-heads, loading its 8 rows together; the
-// 8 x GRP dot products are summed over the warp with warp_sum_spread, so
-// lane-groups of the warp store the scores of one head's 8 blocks side by side.
+// 8 x GRP dot products are summed over the warp with warp_sum_spread, after
+// which the 8 scores of a head sit in 8 lanes and go to 8 consecutive words.
 template <int D, int GRP>
 __global__ void __launch_bounds__(256) decode_score_kernel(const DecodeParams p) {
   constexpr int PER = D / 32;
